@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Throughput of the tensor-parallel MLP block (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--t T]
+                    [--impl ours|reference]
+
+One step = one forward + one backward of the block (all six GEMMs, the two
+shard reductions and the two bias-gradient column sums) on one batch of
+seeded synthetic input already resident in HBM.  The metric is algorithmic
+TFLOP/s, 12·T·h·f per step.  With N > 1 (one process per GPU under
+torchrun) every rank runs an independent replica on its own batch (weak
+scaling, no collective on the data path); `value` is all ranks' FLOPs over
+the slowest rank's device time.
+
+Rank 0 prints one JSON line.  Besides the device-resident number it reports
+`e2e` (the same metric through the public entry points with the step's
+inputs copied from pinned host memory and its outputs copied back inside the
+timed region), `roofline` for the dominant kernel, `cpu_baseline` (the fp64
+oracle timed on this host's cores on a bounded sample), the GPU clocks seen
+during the timed region and the number of library kernel launches in it.
+
+--impl reference times the fp64 CPU oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "TP-sharded MLP fwd+bwd TFLOP/s on 1 B200 and % of dense BF16 peak"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0  # NVIDIA B200 datasheet, dense (non-sparse) BF16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ("fc1_forward", "fc2_forward", "fc2_backward_data", "fc2_backward_weight",
+          "fc1_backward_data", "fc1_backward_weight")
+STAGE_KERNEL = {
+    "fc1_forward": "Z=X·A+a, H=GeLU(Z) (column-parallel GEMM, bias+GeLU epilogue)",
+    "fc2_forward": "Y=Σ_i H_i·B_i + b (row-parallel GEMM, shard-sum epilogue)",
+    "fc2_backward_data": "dH=(dY·Bᵀ)⊙GeLU'(Z) (GEMM, GeLU-derivative epilogue)",
+    "fc2_backward_weight": "dB=Hᵀ·dY (GEMM) + db column sum",
+    "fc1_backward_data": "dX=Σ_i dH_i·A_iᵀ (GEMM, shard-sum epilogue)",
+    "fc1_backward_weight": "dA=Xᵀ·dH (GEMM) + da column sum",
+}
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max_sum(local_ms: float, local_units: float, group=None):
+    """Max of the per-rank device times and sum of the per-rank work, over all
+    ranks (identity when torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return local_ms, local_units
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([local_units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), float(u.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        loaded = [s for s in sm if mx and s >= 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()),
+                                   default=None)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample_step(inp, rows):
+    """One forward+backward of the fp64 oracle on the first `rows` tokens."""
+    from oracle import mlp_oracle
+    X = inp["X"][:rows]
+    dY = inp["dY"][:rows]
+    mlp_oracle.forward(X, inp["A"], inp["a"], inp["B"], inp["b"])
+    mlp_oracle.backward(dY, X, inp["A"], inp["a"], inp["B"])
+
+
+def calibrate_oracle_rows(inp, wl, target_s):
+    rows = min(wl.T, 16)
+    t0 = time.perf_counter()
+    oracle_sample_step(inp, rows)
+    dt = time.perf_counter() - t0
+    scaled = int(rows * target_s / max(dt, 1e-3))
+    return max(16, min(wl.T, scaled))
+
+
+def cpu_baseline(inp, wl, target_s=12.0):
+    rows = calibrate_oracle_rows(inp, wl, target_s)
+    t0 = time.perf_counter()
+    oracle_sample_step(inp, rows)
+    dt = time.perf_counter() - t0
+    fl = 12.0 * rows * wl.h * wl.f
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, forward+backward of the first {rows} of {wl.T} tokens with the full "
+                      f"h={wl.h} x f={wl.f} weights ({fl:.3g} FLOPs, {dt:.1f} s)"}
+
+
+def run_reference(args, wl, ws, rank):
+    """Reference arm: the fp64 CPU oracle, as it stands, on bounded samples."""
+    if rank != 0:
+        return 0
+    from tensor_transformer_mlp_bias_b200 import inputs
+    inp = inputs.make_inputs(wl)
+    per_step_s = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = calibrate_oracle_rows(inp, wl, per_step_s)
+    for _ in range(args.warmup):
+        oracle_sample_step(inp, rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_sample_step(inp, rows)
+        times.append(time.perf_counter() - t0)
+    fl = 12.0 * rows * wl.h * wl.f
+    total = sum(times)
+    value = fl * len(times) / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Gaussian, bf16-rounded, upcast to fp64)",
+        "config": workload_config(wl, args.t, ws),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: forward+backward of the first {rows} of {wl.T} tokens, full weights"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, t, ws):
+    return {"workload": f"{wl.name} MLP block: T={wl.T} tokens, h={wl.h}, f={wl.f}, t={t} shards on one GPU",
+            "T": wl.T, "h": wl.h, "f": wl.f, "t": t, "flops_per_step": wl.flops,
+            "parallelism": f"replicas x{ws} (t shards per GPU reduced on device)",
+            "l2": "inputs larger than L2 (A and B are h*f*2 bytes each; no flush)"}
+
+
+# ---------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="h4096")
+    ap.add_argument("--t", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    from tensor_transformer_mlp_bias_b200 import inputs
+    wl = inputs.WORKLOADS[args.workload]
+    if args.t is None:
+        args.t = max(wl.shards)
+    world, rank, local = dist_env()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return run_reference(args, wl, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    from tensor_transformer_mlp_bias_b200 import binding
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    binding.lib()
+
+    T, h, f, t = wl.T, wl.h, wl.f, args.t
+    host = inputs.make_inputs(wl, seed=wl.seed + rank)
+    dev = {k: v.cuda() for k, v in host.items()}
+    e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
+    Z, H, Y, dH = e(T, f), e(T, f), e(T, h), e(T, f)
+    dX, dA, dB, da, db = e(T, h), e(h, f), e(f, h), e(f), e(h)
+    ws = binding.make_workspace(T, h, f, t)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step(evs=None):
+        calls = (
+            lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, ws, sh),
+            lambda: binding.mlp_tp_fc2_forward(H, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_weight(H, dev["dY"], T, h, f, t, dB, db, ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_data(dH, dev["A"], T, h, f, t, dX, ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], dH, T, h, f, t, dA, da, ws, sh),
+        )
+        for i, c in enumerate(calls):
+            if evs is not None:
+                evs[i].record(stream)
+            c()
+        if evs is not None:
+            evs[len(calls)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    binding.mlp_tp_check(ws, sh)
+
+    # ------------------------------------------------ device-resident timing
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        l0 = binding.mlp_tp_launch_count()
+        start.record(stream)
+        for k in range(args.steps):
+            step(ev[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+        launches = binding.mlp_tp_launch_count() - l0
+    if world > 1:
+        dist.barrier()
+    binding.mlp_tp_check(ws, sh)
+    local_ms = start.elapsed_time(end)
+    stage_ms = {s: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps))
+                for i, s in enumerate(STAGES)}
+    max_ms, total_flops = reduce_max_sum(local_ms, float(wl.flops) * args.steps)
+    value = total_flops / (max_ms * 1e-3) / 1e12
+    ms_per_step = max_ms / args.steps
+
+    # ------------------------------------------------ end-to-end through the public API
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    outs_host = {"Y": torch.empty(T, h, dtype=torch.bfloat16).pin_memory(),
+                 "dX": torch.empty(T, h, dtype=torch.bfloat16).pin_memory(),
+                 "dA": torch.empty(h, f, dtype=torch.bfloat16).pin_memory(),
+                 "da": torch.empty(f, dtype=torch.bfloat16).pin_memory(),
+                 "dB": torch.empty(f, h, dtype=torch.bfloat16).pin_memory(),
+                 "db": torch.empty(h, dtype=torch.bfloat16).pin_memory()}
+    outs_dev = {"Y": Y, "dX": dX, "dA": dA, "da": da, "dB": dB, "db": db}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
+
+    def e2e_step():
+        for k, v in pin.items():
+            dev[k].copy_(v, non_blocking=True)
+        binding.mlp_tp_forward(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, Y, Z, H, ws, sh)
+        binding.mlp_tp_backward(dev["dY"], dev["X"], dev["A"], dev["B"], Z, H, T, h, f, t,
+                                dX, dA, da, dB, db, ws, sh)
+        for k, v in outs_host.items():
+            v.copy_(outs_dev[k], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    binding.mlp_tp_check(ws, sh)
+    e2e_ms, e2e_flops = reduce_max_sum(s2.elapsed_time(e2), float(wl.flops) * args.e2e_steps)
+    e2e_value = e2e_flops / (e2e_ms * 1e-3) / 1e12
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # ------------------------------------------------ roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    dom = max(STAGES, key=lambda s: stage_ms[s])
+    gemm_flops = 2.0 * T * h * f
+    achieved = gemm_flops / (stage_ms[dom] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    roofline = {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved,
+                "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "traffic": traffic_for(dom, wl, t),
+                "algorithmic_flops_per_launch": gemm_flops, "avg_launch_ms": stage_ms[dom]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, bf16)",
+        "config": workload_config(wl, t, world),
+        "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_DENSE_TFLOPS,
+        "pct_of_measured_bf16_peak": 100.0 * value / world / float(peaks.get("bf16_tflops", 1713.1)),
+        "stage_ms": stage_ms,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps, "api": "mlp_tp_forward + mlp_tp_backward, pinned host buffers"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(host, wl)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def traffic_for(stage, wl, t):
+    """DRAM bytes per launch of the stage's kernel from the committed ncu
+    summary, when it was captured for this workload and the kernel source has
+    not changed since (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = kernel_source_digest()
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) >= 5 and not ln.startswith("#") and parts[0] == stage and parts[1] == wl.name \
+                and parts[2] == f"t={t}" and parts[3] == src:
+            return float(parts[4])
+    return None
+
+
+def kernel_source_digest():
+    import hashlib
+    hsh = hashlib.sha256()
+    for n in ("gemm.cuh", "ptx.cuh", "colsum.cuh", "mlp_tp.cu"):
+        with open(os.path.join(ROOT, "tensor_transformer_mlp_bias_b200", "csrc", n), "rb") as fh:
+            hsh.update(fh.read())
+    return hsh.hexdigest()[:12]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,180 @@
+/*
+ * mlp_tp.h — C-ABI of the B200 (sm_100a) tensor-parallel Transformer MLP block
+ * with biases, all t shards on one GPU.
+ *
+ *   forward   Y = sum_{i<t} GeLU(X·A_i + a_i)·B_i + b
+ *   backward  dX, dA, da, dB, db given dY
+ *
+ * The block is Megatron's Column->Row parallel MLP: the first linear layer's
+ * weight A[h,f] is split by columns into A_i (ColumnParallelLinear, output not
+ * gathered), the second layer's weight B[f,h] by rows into B_i
+ * (RowParallelLinear, input already parallel), and the t partial outputs are
+ * summed once ("Megatron-LM — 架构与原理", §4 巧妙之处, item "Column→Row 配对让
+ * MLP 只做一次通信"; "Megatron-LM（英伟达超大模型训练框架）完整介绍", §二.2 MLP层).
+ * The all-reduce of the forward ("reduce" operator) and of the backward
+ * ("copy" operator's backward, same §4, item "通信原语的「前向/反向对偶」") become
+ * on-device shard reductions: Y = P_0 + P_1 + ... + P_{t-1} + b and
+ * dX = Q_0 + ... + Q_{t-1}, summed in fp32 in ascending shard order and
+ * rounded once to bf16.  GeLU is the tanh form
+ * g(x) = x/2·(1 + tanh(sqrt(2/pi)·(x + 0.044715·x^3))).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All matrices are row-major, contiguous, bf16 (IEEE bfloat16), in device
+ *    memory owned by the caller: X[T,h], A[h,f], a[f], B[f,h], b[h],
+ *    Z[T,f], H[T,f], Y[T,h], dY[T,h], dH[T,f], dX[T,h], dA[h,f], da[f],
+ *    dB[f,h], db[h].  Shard i owns columns [i·f/t, (i+1)·f/t) of A, a, Z, H,
+ *    dH, dA, da and rows [i·f/t, (i+1)·f/t) of B and dB.
+ *  - Every device pointer must be 16-byte aligned.  Inputs are only read;
+ *    outputs are overwritten (never accumulated into).  Outputs must not
+ *    alias inputs or each other.
+ *  - Shapes: T >= 0, h >= 64 and h % 64 == 0, t >= 1, f % t == 0,
+ *    fs = f/t >= 64 and fs % 64 == 0, and T, h, f < 2^31.
+ *  - `ws` is a caller-owned device workspace of at least
+ *    mlp_tp_workspace_bytes(T, h, f, t) bytes, zero-filled once before its
+ *    first use; the library keeps a device status word in its first bytes
+ *    and scratch after it.  Calls that share a workspace must be ordered on
+ *    one stream.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; no entry point except mlp_tp_check synchronises, and
+ *    none allocates or frees memory.
+ *  - Arguments are validated on the host before anything is launched; on any
+ *    error nothing is enqueued.  Errors raised by the CUDA runtime when
+ *    launching map to MLP_ERR_CUDA.  Faults found by the kernels themselves
+ *    (a bounded wait that ran out) are reported by mlp_tp_check.
+ *  - The current CUDA device must be an sm_100 part (B200); there is no other
+ *    code path and no CPU fallback.
+ */
+#ifndef MLP_TP_H_
+#define MLP_TP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLP_OK = 0,
+  MLP_ERR_INVALID_ARG = 1,         /* null pointer, negative size, t < 1 */
+  MLP_ERR_UNSUPPORTED_SHAPE = 2,   /* divisibility / range rules above violated */
+  MLP_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
+  MLP_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < mlp_tp_workspace_bytes(...) */
+  MLP_ERR_UNSUPPORTED_DEVICE = 5,  /* current device is not sm_100, or none */
+  MLP_ERR_CUDA = 6,                /* the CUDA runtime reported an error */
+  MLP_ERR_TIMEOUT = 7              /* a kernel's bounded wait ran out (mlp_tp_check) */
+} mlp_status_t;
+
+/* Bytes of workspace needed by every entry point below for this shape
+ * (the maximum over all of them): a 256-byte status header, the dH buffer
+ * used by mlp_tp_backward, and fp32 column-sum partials.  Returns 0 for an
+ * invalid shape. */
+size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
+
+/* ---------------------------------------------------------------- forward */
+
+/* Whole forward: mlp_tp_fc1_forward then mlp_tp_fc2_forward.
+ * Writes Y[T,h] and saves Z[T,f] = X·A + a and H[T,f] = g(Z) for the
+ * backward. */
+mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a,
+                            const void* B, const void* b,
+                            int64_t T, int64_t h, int64_t f, int32_t t,
+                            void* Y, void* Z, void* H,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ColumnParallelLinear of every shard plus the activation:
+ * Z_i = X·A_i + a_i and H_i = g(Z_i), for all i in one launch (shard i is
+ * the column block i of Z and H).  No reduction: the column split needs
+ * none. */
+mlp_status_t mlp_tp_fc1_forward(const void* X, const void* A, const void* a,
+                                int64_t T, int64_t h, int64_t f, int32_t t,
+                                void* Z, void* H,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* RowParallelLinear of every shard plus the reduce that stands in for the
+ * forward all-reduce: P_i = H_i·B_i in fp32, Y = (((P_0 + P_1) + ...) +
+ * P_{t-1}) + b, rounded once to bf16.  `b` may be NULL (no bias). */
+mlp_status_t mlp_tp_fc2_forward(const void* H, const void* B, const void* b,
+                                int64_t T, int64_t h, int64_t f, int32_t t,
+                                void* Y,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------- backward */
+
+/* Whole backward, given dY and the Z, H saved by the forward:
+ * mlp_tp_fc2_backward_data (dH into the workspace), mlp_tp_fc2_backward_weight,
+ * mlp_tp_fc1_backward_data and mlp_tp_fc1_backward_weight.
+ * `da` and `db` may be NULL (bias gradients not wanted). */
+mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A,
+                             const void* B, const void* Z, const void* H,
+                             int64_t T, int64_t h, int64_t f, int32_t t,
+                             void* dX, void* dA, void* da, void* dB, void* db,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of the row-parallel layer through the activation, per shard:
+ * dH_i = (dY·B_iᵀ) ⊙ g'(Z_i).  dY reaches every shard unchanged (the
+ * reduce's backward is the identity).  Writes dH[T,f]. */
+mlp_status_t mlp_tp_fc2_backward_data(const void* dY, const void* B, const void* Z,
+                                      int64_t T, int64_t h, int64_t f, int32_t t,
+                                      void* dH,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* Weight gradients of the row-parallel layer: dB_i = H_iᵀ·dY (each shard's
+ * own rows of dB, no reduction) and db = sum over rows of dY (NULL: skip). */
+mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* dY,
+                                        int64_t T, int64_t h, int64_t f, int32_t t,
+                                        void* dB, void* db,
+                                        void* ws, size_t ws_bytes, void* stream);
+
+/* Input gradient of the column-parallel layer plus the reduce that stands in
+ * for the copy operator's backward all-reduce: Q_i = dH_i·A_iᵀ in fp32,
+ * dX = ((Q_0 + Q_1) + ...) + Q_{t-1}, rounded once to bf16. */
+mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* A,
+                                      int64_t T, int64_t h, int64_t f, int32_t t,
+                                      void* dX,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* Weight gradients of the column-parallel layer: dA_i = Xᵀ·dH_i (each
+ * shard's own columns of dA) and da = sum over rows of dH (NULL: skip). */
+mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH,
+                                        int64_t T, int64_t h, int64_t f, int32_t t,
+                                        void* dA, void* da,
+                                        void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+/* Synchronises `stream`, then reads and clears the device status word in
+ * `ws`.  Returns MLP_OK, MLP_ERR_TIMEOUT (a kernel's bounded wait ran out;
+ * its outputs are undefined, the CUDA context stays usable) or MLP_ERR_CUDA
+ * (the stream reported an error). */
+mlp_status_t mlp_tp_check(void* ws, void* stream);
+
+/* Static, NUL-terminated name of a status code. */
+const char* mlp_tp_status_string(mlp_status_t status);
+
+/* Thread-local, NUL-terminated description of the last error returned to
+ * this thread (which argument, which CUDA call).  Valid until the next call
+ * from the same thread. */
+const char* mlp_tp_last_error(void);
+
+/* Number of kernels the library enqueued from this process so far (all
+ * threads).  Used to count launches inside a timed region. */
+uint64_t mlp_tp_launch_count(void);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel (default
+ * 1e9).  Past it the kernel records MLP_ERR_TIMEOUT and returns.  Applies to
+ * later launches; values below 1e6 are raised to 1e6. */
+void mlp_tp_set_wait_budget_ns(uint64_t ns);
+
+/* Test hook: when `flags` & 1, the next launches' operand-loading warp
+ * stops after its first tile stage, so the tensor-core warp's wait for the
+ * second stage can only end by running out of its budget.  Takes effect on
+ * launches enqueued after the call; 0 restores normal operation. */
+void mlp_tp_set_debug_flags(uint32_t flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLP_TP_H_ */

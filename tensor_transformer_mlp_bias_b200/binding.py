@@ -1,0 +1,211 @@
+"""ctypes binding of the C-ABI library ``libmlptp.so`` (include/mlp_tp.h).
+
+Argument marshalling only: every function here takes torch tensors (or raw
+integer device addresses), checks that tensors are contiguous bf16 CUDA
+tensors, passes their addresses and the stream to the C entry point of the
+same name, and raises :class:`MlpError` on a non-OK status.  All arithmetic
+runs in the library's kernels.  The library is loaded on first use; if it
+has not been built, the call raises (there is no fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmlptp.so")
+
+STATUS = {
+    0: "MLP_OK",
+    1: "MLP_ERR_INVALID_ARG",
+    2: "MLP_ERR_UNSUPPORTED_SHAPE",
+    3: "MLP_ERR_MISALIGNED",
+    4: "MLP_ERR_WORKSPACE_TOO_SMALL",
+    5: "MLP_ERR_UNSUPPORTED_DEVICE",
+    6: "MLP_ERR_CUDA",
+    7: "MLP_ERR_TIMEOUT",
+}
+
+# name -> argument ctypes, in header order
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "mlp_tp_workspace_bytes": ([_I64, _I64, _I64, _I32], _SZ),
+    "mlp_tp_forward": ([_P] * 5 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_forward": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_forward": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_backward": ([_P] * 6 + [_I64, _I64, _I64, _I32] + [_P] * 5 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_weight": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_data": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_weight": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_check": ([_P, _P], ctypes.c_int),
+    "mlp_tp_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "mlp_tp_last_error": ([], ctypes.c_char_p),
+    "mlp_tp_launch_count": ([], ctypes.c_uint64),
+    "mlp_tp_set_wait_budget_ns": ([ctypes.c_uint64], None),
+    "mlp_tp_set_debug_flags": ([ctypes.c_uint32], None),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class MlpError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmlptp.so (once).  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is not built; run `python -m tensor_transformer_mlp_bias_b200.build` "
+                "(the CUDA library is the only implementation; there is no fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+# ------------------------------------------------------------------ marshalling
+def _addr(x, name: str, nullable: bool = False):
+    if x is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if isinstance(x, int):
+        return x
+    import torch
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor or an int address")
+    if x.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {x.device})")
+    if x.dtype != torch.bfloat16 and name != "ws":
+        raise ValueError(f"{name} must be bfloat16 (got {x.dtype})")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ws(ws):
+    import torch
+    if isinstance(ws, torch.Tensor):
+        return _addr(ws, "ws"), ws.numel() * ws.element_size()
+    addr, nbytes = ws
+    return addr, nbytes
+
+
+def _check(status: int):
+    if status != 0:
+        msg = lib().mlp_tp_last_error()
+        raise MlpError(status, msg.decode() if msg else "")
+
+
+def workspace_bytes(T: int, h: int, f: int, t: int) -> int:
+    return int(lib().mlp_tp_workspace_bytes(T, h, f, t))
+
+
+def make_workspace(T: int, h: int, f: int, t: int, device="cuda"):
+    """Zero-filled uint8 device workspace (torch allocations are 256-byte aligned)."""
+    import torch
+    n = workspace_bytes(T, h, f, t)
+    if n == 0:
+        raise MlpError(2, f"unsupported shape T={T} h={h} f={f} t={t}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def mlp_tp_forward(X, A, a, B, b, T, h, f, t, Y, Z, H, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"), _addr(b, "b"),
+                                T, h, f, t, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), T, h, f, t,
+                                    _addr(Z, "Z"), _addr(H, "H"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_forward(H, B, b, T, h, f, t, Y, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_forward(_addr(H, "H"), _addr(B, "B"), _addr(b, "b", True), T, h, f, t,
+                                    _addr(Y, "Y"), w, wn, _stream(stream)))
+
+
+def mlp_tp_backward(dY, X, A, B, Z, H, T, h, f, t, dX, dA, da, dB, db, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_backward(_addr(dY, "dY"), _addr(X, "X"), _addr(A, "A"), _addr(B, "B"), _addr(Z, "Z"),
+                                 _addr(H, "H"), T, h, f, t, _addr(dX, "dX"), _addr(dA, "dA"),
+                                 _addr(da, "da", True), _addr(dB, "dB"), _addr(db, "db", True), w, wn,
+                                 _stream(stream)))
+
+
+def mlp_tp_fc2_backward_data(dY, B, Z, T, h, f, t, dH, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_backward_data(_addr(dY, "dY"), _addr(B, "B"), _addr(Z, "Z"), T, h, f, t,
+                                          _addr(dH, "dH"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_backward_weight(H, dY, T, h, f, t, dB, db, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_backward_weight(_addr(H, "H"), _addr(dY, "dY"), T, h, f, t, _addr(dB, "dB"),
+                                            _addr(db, "db", True), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_data(dH, A, T, h, f, t, dX, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_data(_addr(dH, "dH"), _addr(A, "A"), T, h, f, t, _addr(dX, "dX"),
+                                          w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_weight(X, dH, T, h, f, t, dA, da, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_weight(_addr(X, "X"), _addr(dH, "dH"), T, h, f, t, _addr(dA, "dA"),
+                                            _addr(da, "da", True), w, wn, _stream(stream)))
+
+
+def mlp_tp_check(ws, stream=None):
+    w, _ = _ws(ws)
+    _check(lib().mlp_tp_check(w, _stream(stream)))
+
+
+def mlp_tp_status_string(status: int) -> str:
+    return lib().mlp_tp_status_string(status).decode()
+
+
+def mlp_tp_last_error() -> str:
+    return lib().mlp_tp_last_error().decode()
+
+
+def mlp_tp_launch_count() -> int:
+    return int(lib().mlp_tp_launch_count())
+
+
+def mlp_tp_set_wait_budget_ns(ns: int):
+    lib().mlp_tp_set_wait_budget_ns(ns)
+
+
+def mlp_tp_set_debug_flags(flags: int):
+    lib().mlp_tp_set_debug_flags(flags)

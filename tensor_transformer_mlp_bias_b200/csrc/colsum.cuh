@@ -1,0 +1,74 @@
+// Column sums of a row-major bf16 matrix M[R, C] in fp32, in a fixed order:
+// the bias gradients da = Σ_rows dH and db = Σ_rows dY.
+//
+// Pass 1 (colsum_partial): block (32, 8); thread x owns 8 consecutive
+// columns (one 16-byte load per row, so a warp reads 512 contiguous bytes of
+// a row); thread y walks rows y, y+8, ... of a chunk of ROWS_PER_CHUNK rows.
+// The 8 row phases are combined through shared memory in ascending order and
+// the chunk's partial sums are written to the fp32 scratch [chunks, C].
+// Pass 2 (colsum_final): one thread per column adds the chunk partials in
+// ascending chunk order and rounds once to bf16.  The result is therefore
+// deterministic and independent of the launch configuration's timing.
+// Both passes are HBM-bound: R·C·2 bytes read once.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace mlptp {
+
+constexpr int COLSUM_ROWS_PER_CHUNK = 256;
+constexpr int COLSUM_COLS_PER_BLOCK = 32 * 8;
+
+__global__ void __launch_bounds__(256) colsum_partial(const __nv_bfloat16* __restrict__ m, int R, int C,
+                                                      float* __restrict__ partial) {
+  __shared__ float red[8][32][9];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int c0 = (blockIdx.x * 32 + tx) * 8;
+  const int r_begin = blockIdx.y * COLSUM_ROWS_PER_CHUNK;
+  const int r_end = min(R, r_begin + COLSUM_ROWS_PER_CHUNK);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  if (c0 < C) {
+    const __nv_bfloat16* base = m + c0;
+    for (int r = r_begin + ty; r < r_end; r += 8) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * C));
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
+        const float2 f = __bfloat1622float2(b2);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[ty][tx][e] = acc[e];
+  __syncthreads();
+  if (ty == 0 && c0 < C) {
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float s = red[0][tx][e];
+#pragma unroll
+      for (int y = 1; y < 8; ++y) s += red[y][tx][e];
+      out[e] = s;
+    }
+    float4* dst = reinterpret_cast<float4*>(partial + static_cast<size_t>(blockIdx.y) * C + c0);
+    dst[0] = make_float4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+__global__ void __launch_bounds__(256) colsum_final(const float* __restrict__ partial, int chunks, int C,
+                                                    __nv_bfloat16* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  float s = 0.0f;
+  for (int k = 0; k < chunks; ++k) s += partial[static_cast<size_t>(k) * C + c];
+  out[c] = __float2bfloat16_rn(s);
+}
+
+}  // namespace mlptp

@@ -1,0 +1,501 @@
+// C-ABI of the tensor-parallel MLP block (declared in include/mlp_tp.h):
+// host-side validation, TMA descriptor construction and kernel launches.
+// Nothing here allocates device memory or synchronises, except mlp_tp_check.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mlp_tp.h"
+#include "colsum.cuh"
+#include "gemm.cuh"
+
+using namespace mlptp;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_budget_ns{1000000000ull};
+std::atomic<uint32_t> g_debug_flags{0};
+
+constexpr size_t WS_HEADER_BYTES = 256;
+
+mlp_status_t fail(mlp_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+mlp_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(MLP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- shapes
+struct Shape {
+  int64_t T, h, f;
+  int32_t t;
+  int64_t fs() const { return f / t; }
+};
+
+mlp_status_t check_shape(const Shape& s) {
+  if (s.T < 0 || s.h < 0 || s.f < 0) return fail(MLP_ERR_INVALID_ARG, "negative size T=%lld h=%lld f=%lld",
+                                                 (long long)s.T, (long long)s.h, (long long)s.f);
+  if (s.t < 1) return fail(MLP_ERR_INVALID_ARG, "shard count t=%d must be >= 1", s.t);
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (s.T > lim || s.h > lim || s.f > lim)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "T, h and f must be < 2^31");
+  if (s.h < 64 || s.h % 64 != 0) return fail(MLP_ERR_UNSUPPORTED_SHAPE, "h=%lld must be a positive multiple of 64",
+                                             (long long)s.h);
+  if (s.f % s.t != 0) return fail(MLP_ERR_UNSUPPORTED_SHAPE, "f=%lld is not divisible by t=%d", (long long)s.f, s.t);
+  if (s.fs() < 64 || s.fs() % 64 != 0)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "shard width f/t=%lld must be a positive multiple of 64",
+                (long long)s.fs());
+  return MLP_OK;
+}
+
+size_t colsum_chunks(int64_t R) { return static_cast<size_t>((R + COLSUM_ROWS_PER_CHUNK - 1) / COLSUM_ROWS_PER_CHUNK); }
+
+size_t dh_offset() { return WS_HEADER_BYTES; }
+size_t partial_offset(const Shape& s) { return WS_HEADER_BYTES + align_up(static_cast<size_t>(s.T * s.f * 2), 256); }
+size_t workspace_bytes(const Shape& s) {
+  const size_t cols = static_cast<size_t>(s.f > s.h ? s.f : s.h);
+  return partial_offset(s) + align_up(colsum_chunks(s.T) * cols * sizeof(float), 256);
+}
+
+struct Ptr {
+  const void* p;
+  const char* name;
+  bool nullable;
+};
+
+mlp_status_t check_ptrs(std::initializer_list<Ptr> ptrs) {
+  for (const Ptr& x : ptrs) {
+    if (x.p == nullptr) {
+      if (x.nullable) continue;
+      return fail(MLP_ERR_INVALID_ARG, "pointer %s is NULL", x.name);
+    }
+    if (reinterpret_cast<uintptr_t>(x.p) % 16 != 0)
+      return fail(MLP_ERR_MISALIGNED, "pointer %s is not 16-byte aligned", x.name);
+  }
+  return MLP_OK;
+}
+
+mlp_status_t check_ws(const Shape& s, void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MLP_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+  const size_t need = workspace_bytes(s);
+  if (ws_bytes < need)
+    return fail(MLP_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return MLP_OK;
+}
+
+// ---------------------------------------------------------------- device
+struct DeviceInfo {
+  bool probed = false;
+  bool ok = false;
+  int sms = 0;
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+mlp_status_t current_device(int& dev, int& sms) {
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MLP_ERR_UNSUPPORTED_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(MLP_ERR_UNSUPPORTED_DEVICE, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return fail(MLP_ERR_UNSUPPORTED_DEVICE, "cannot query device %d", dev);
+    d.ok = (major == 10 && minor == 0);
+    d.probed = true;
+    if (!d.ok) return fail(MLP_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d%d; this library runs on sm_100 only", dev,
+                           major, minor);
+  }
+  if (!d.ok) return fail(MLP_ERR_UNSUPPORTED_DEVICE, "device %d is not sm_100", dev);
+  sms = d.sms;
+  return MLP_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major matrix [rows, cols] (cols contiguous), box of
+// 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, uint32_t box_rows,
+                      const char* name) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for %s (CUresult %d)", name, (int)r);
+  return MLP_OK;
+}
+
+// Operand of the GEMM: `rows` is its M (or N) extent, `k` its K extent.
+// K-major: stored [rows, k];  MN-major: stored [k, rows].
+mlp_status_t make_operand_map(CUtensorMap* map, const void* ptr, bool mn_major, int64_t rows, int64_t k,
+                              uint32_t tile_rows, const char* name) {
+  if (mn_major) return make_map(map, ptr, k, rows, 64u, name);
+  return make_map(map, ptr, rows, k, tile_rows, name);
+}
+
+// ---------------------------------------------------------------- launches
+struct GemmDesc {
+  const void* a;  // Aop
+  bool a_mn;
+  const void* b;  // Bop
+  bool b_mn;
+  int64_t M, N, K;  // K = shards * kseg
+  int shards;
+};
+
+int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
+  const double l2_share = 48.0 * 1024 * 1024;
+  const double a_bytes = double(M) * double(K) * 2.0, b_bytes = double(N) * double(K) * 2.0;
+  if (a_bytes <= l2_share) return m_blocks;  // row operand stays resident; walk rows fastest
+  if (b_bytes <= l2_share) return 1;         // column operand stays resident; walk columns fastest
+  return m_blocks < 16 ? m_blocks : 16;
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, int sms, cudaStream_t stream, const char* name) {
+  if (g.M == 0 || g.N == 0) return MLP_OK;
+  CUtensorMap ma, mb;
+  mlp_status_t st = make_operand_map(&ma, g.a, A_MN, g.M, g.K, BM, name);
+  if (st != MLP_OK) return st;
+  st = make_operand_map(&mb, g.b, B_MN, g.N, g.K, BN, name);
+  if (st != MLP_OK) return st;
+
+  p.M = static_cast<int>(g.M);
+  p.N = static_cast<int>(g.N);
+  p.shards = g.shards;
+  p.kblocks_per_shard = static_cast<int>((g.K / g.shards + BK - 1) / BK);
+  p.m_blocks = static_cast<int>((g.M + BM - 1) / BM);
+  p.n_blocks = static_cast<int>((g.N + BN - 1) / BN);
+  p.num_tiles = p.m_blocks * p.n_blocks;
+  p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
+  p.budget_ns = g_budget_ns.load();
+  p.debug_flags = g_debug_flags.load();
+
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(mlp_gemm_kernel<A_MN, B_MN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    GEMM_SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(max dynamic shared memory)");
+
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  mlp_gemm_kernel<A_MN, B_MN, EPI><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, stream>>>(ma, mb, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float* partial, cudaStream_t stream) {
+  if (R == 0) {
+    cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(C) * 2, stream);
+    return e == cudaSuccess ? MLP_OK : cuda_fail(e, "cudaMemsetAsync(bias gradient)");
+  }
+  const int chunks = static_cast<int>(colsum_chunks(R));
+  dim3 grid1(static_cast<unsigned>((C + COLSUM_COLS_PER_BLOCK - 1) / COLSUM_COLS_PER_BLOCK), chunks);
+  colsum_partial<<<grid1, dim3(32, 8), 0, stream>>>(static_cast<const __nv_bfloat16*>(m), static_cast<int>(R),
+                                                    static_cast<int>(C), partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "colsum_partial");
+  g_launches.fetch_add(1);
+  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(partial, chunks, static_cast<int>(C),
+                                                                           static_cast<__nv_bfloat16*>(out));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "colsum_final");
+  g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+GemmParams base_params(void* ws) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.status = static_cast<unsigned int*>(ws);
+  return p;
+}
+
+// ---------------------------------------------------------------- stages
+mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H, void* ws,
+                         int sms, cudaStream_t st) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(Z);
+  p.out1 = static_cast<__nv_bfloat16*>(H);
+  p.bias = static_cast<const __nv_bfloat16*>(a);
+  GemmDesc g{X, false, A, true, s.T, s.f, s.h, 1};
+  return launch_gemm<false, true, EPI_BIAS_GELU>(g, p, sms, st, "column-parallel forward (Z, H)");
+}
+
+mlp_status_t fc2_forward(const Shape& s, const void* H, const void* B, const void* b, void* Y, void* ws, int sms,
+                         cudaStream_t st) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(Y);
+  p.bias = static_cast<const __nv_bfloat16*>(b);
+  GemmDesc g{H, false, B, true, s.T, s.h, s.f, s.t};
+  return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, sms, st, "row-parallel forward + shard reduce (Y)");
+}
+
+mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, const void* Z, void* dH, void* ws,
+                               int sms, cudaStream_t st) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dH);
+  p.aux = static_cast<const __nv_bfloat16*>(Z);
+  GemmDesc g{dY, false, B, false, s.T, s.f, s.h, 1};
+  return launch_gemm<false, false, EPI_GELU_GRAD>(g, p, sms, st, "row-parallel backward data (dH)");
+}
+
+mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* dY, void* dB, void* db, void* ws,
+                                 int sms, cudaStream_t st) {
+  if (s.T == 0) {
+    cudaError_t e = cudaMemsetAsync(dB, 0, static_cast<size_t>(s.f * s.h * 2), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dB)");
+  } else {
+    GemmParams p = base_params(ws);
+    p.out0 = static_cast<__nv_bfloat16*>(dB);
+    GemmDesc g{H, true, dY, true, s.f, s.h, s.T, 1};
+    mlp_status_t r = launch_gemm<true, true, EPI_STORE>(g, p, sms, st, "row-parallel weight gradient (dB)");
+    if (r != MLP_OK) return r;
+  }
+  if (db == nullptr) return MLP_OK;
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
+  return launch_colsum(dY, s.T, s.h, db, partial, st);
+}
+
+mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* A, void* dX, void* ws, int sms,
+                               cudaStream_t st) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dX);
+  GemmDesc g{dH, false, A, false, s.T, s.h, s.f, s.t};
+  return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, sms, st, "column-parallel backward data + shard reduce (dX)");
+}
+
+mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, void* dA, void* da, void* ws, int sms,
+                                 cudaStream_t st) {
+  if (s.T == 0) {
+    cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(s.h * s.f * 2), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dA)");
+  } else {
+    GemmParams p = base_params(ws);
+    p.out0 = static_cast<__nv_bfloat16*>(dA);
+    GemmDesc g{X, true, dH, true, s.h, s.f, s.T, 1};
+    mlp_status_t r = launch_gemm<true, true, EPI_STORE>(g, p, sms, st, "column-parallel weight gradient (dA)");
+    if (r != MLP_OK) return r;
+  }
+  if (da == nullptr) return MLP_OK;
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
+  return launch_colsum(dH, s.T, s.f, da, partial, st);
+}
+
+// Common preamble: shape, pointers, workspace, device.
+mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, int& sms) {
+  mlp_status_t st = check_shape(s);
+  if (st != MLP_OK) return st;
+  st = check_ptrs(ptrs);
+  if (st != MLP_OK) return st;
+  st = check_ws(s, ws, ws_bytes);
+  if (st != MLP_OK) return st;
+  int dev = 0;
+  return current_device(dev, sms);
+}
+
+}  // namespace
+
+// ====================================================================== C-ABI
+extern "C" {
+
+size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t) {
+  Shape s{T, h, f, t};
+  std::string saved = g_last_error;
+  const bool ok = check_shape(s) == MLP_OK;
+  g_last_error = saved;
+  return ok ? workspace_bytes(s) : 0;
+}
+
+mlp_status_t mlp_tp_fc1_forward(const void* X, const void* A, const void* a, int64_t T, int64_t h, int64_t f,
+                                int32_t t, void* Z, void* H, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st = prologue(s, {{X, "X", false}, {A, "A", false}, {a, "a", false}, {Z, "Z", false}, {H, "H", false}},
+                             ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc1_forward(s, X, A, a, Z, H, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_fc2_forward(const void* H, const void* B, const void* b, int64_t T, int64_t h, int64_t f,
+                                int32_t t, void* Y, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st = prologue(s, {{H, "H", false}, {B, "B", false}, {b, "b", true}, {Y, "Y", false}}, ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc2_forward(s, H, B, b, Y, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a, const void* B, const void* b, int64_t T,
+                            int64_t h, int64_t f, int32_t t, void* Y, void* Z, void* H, void* ws, size_t ws_bytes,
+                            void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st = prologue(s,
+                             {{X, "X", false},
+                              {A, "A", false},
+                              {a, "a", false},
+                              {B, "B", false},
+                              {b, "b", false},
+                              {Y, "Y", false},
+                              {Z, "Z", false},
+                              {H, "H", false}},
+                             ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  st = fc1_forward(s, X, A, a, Z, H, ws, sms, cs);
+  if (st != MLP_OK) return st;
+  return fc2_forward(s, H, B, b, Y, ws, sms, cs);
+}
+
+mlp_status_t mlp_tp_fc2_backward_data(const void* dY, const void* B, const void* Z, int64_t T, int64_t h, int64_t f,
+                                      int32_t t, void* dH, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st =
+      prologue(s, {{dY, "dY", false}, {B, "B", false}, {Z, "Z", false}, {dH, "dH", false}}, ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc2_backward_data(s, dY, B, Z, dH, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* dY, int64_t T, int64_t h, int64_t f, int32_t t,
+                                        void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st =
+      prologue(s, {{H, "H", false}, {dY, "dY", false}, {dB, "dB", false}, {db, "db", true}}, ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc2_backward_weight(s, H, dY, dB, db, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* A, int64_t T, int64_t h, int64_t f, int32_t t,
+                                      void* dX, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st = prologue(s, {{dH, "dH", false}, {A, "A", false}, {dX, "dX", false}}, ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc1_backward_data(s, dH, A, dX, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, int64_t T, int64_t h, int64_t f, int32_t t,
+                                        void* dA, void* da, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st =
+      prologue(s, {{X, "X", false}, {dH, "dH", false}, {dA, "dA", false}, {da, "da", true}}, ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  return fc1_backward_weight(s, X, dH, dA, da, ws, sms, static_cast<cudaStream_t>(stream));
+}
+
+mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const void* B, const void* Z, const void* H,
+                             int64_t T, int64_t h, int64_t f, int32_t t, void* dX, void* dA, void* da, void* dB,
+                             void* db, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  int sms = 0;
+  mlp_status_t st = prologue(s,
+                             {{dY, "dY", false},
+                              {X, "X", false},
+                              {A, "A", false},
+                              {B, "B", false},
+                              {Z, "Z", false},
+                              {H, "H", false},
+                              {dX, "dX", false},
+                              {dA, "dA", false},
+                              {da, "da", true},
+                              {dB, "dB", false},
+                              {db, "db", true}},
+                             ws, ws_bytes, sms);
+  if (st != MLP_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  void* dH = static_cast<char*>(ws) + dh_offset();
+  if ((st = fc2_backward_data(s, dY, B, Z, dH, ws, sms, cs)) != MLP_OK) return st;
+  if ((st = fc2_backward_weight(s, H, dY, dB, db, ws, sms, cs)) != MLP_OK) return st;
+  if ((st = fc1_backward_data(s, dH, A, dX, ws, sms, cs)) != MLP_OK) return st;
+  return fc1_backward_weight(s, X, dH, dA, da, ws, sms, cs);
+}
+
+mlp_status_t mlp_tp_check(void* ws, void* stream) {
+  if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word[2] = {0u, 0u};
+  e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status word");
+  if (word[0] == 0u) return MLP_OK;
+  const unsigned int zero[2] = {0u, 0u};
+  e = cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace status word");
+  if (word[0] == STATUS_TIMEOUT)
+    return fail(MLP_ERR_TIMEOUT, "a kernel wait ran out of its budget (site 0x%x)", word[1]);
+  return fail(MLP_ERR_CUDA, "device status word holds unknown code %u", word[0]);
+}
+
+const char* mlp_tp_status_string(mlp_status_t status) {
+  switch (status) {
+    case MLP_OK: return "MLP_OK";
+    case MLP_ERR_INVALID_ARG: return "MLP_ERR_INVALID_ARG";
+    case MLP_ERR_UNSUPPORTED_SHAPE: return "MLP_ERR_UNSUPPORTED_SHAPE";
+    case MLP_ERR_MISALIGNED: return "MLP_ERR_MISALIGNED";
+    case MLP_ERR_WORKSPACE_TOO_SMALL: return "MLP_ERR_WORKSPACE_TOO_SMALL";
+    case MLP_ERR_UNSUPPORTED_DEVICE: return "MLP_ERR_UNSUPPORTED_DEVICE";
+    case MLP_ERR_CUDA: return "MLP_ERR_CUDA";
+    case MLP_ERR_TIMEOUT: return "MLP_ERR_TIMEOUT";
+  }
+  return "MLP_ERR_UNKNOWN";
+}
+
+const char* mlp_tp_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t mlp_tp_launch_count(void) { return g_launches.load(); }
+
+void mlp_tp_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+void mlp_tp_set_debug_flags(uint32_t flags) { g_debug_flags.store(flags); }
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the
+header declares, and rejects bad arguments on the host before touching the
+device (CPU-only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tensor_transformer_mlp_bias_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mlp_tp.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mlp_tp_\w+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_wraps():
+    assert header_functions() == sorted(binding.exported_symbols())
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert binding.mlp_tp_status_string(code) == name
+
+
+def test_workspace_bytes(lib):
+    n = binding.workspace_bytes(64, 256, 1024, 2)
+    # header 256 + dH 64*1024*2 + one 256-row chunk of max(f,h) fp32 partials
+    assert n == 256 + 64 * 1024 * 2 + 1024 * 4
+    assert binding.workspace_bytes(64, 256, 1000, 2) == 0   # f/t not a multiple of 64
+    assert binding.workspace_bytes(64, 100, 1024, 2) == 0   # h not a multiple of 64
+    assert binding.workspace_bytes(64, 256, 1024, 0) == 0   # t < 1
+    assert binding.workspace_bytes(-1, 256, 1024, 2) == 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned fake address: validation must fail before any use
+
+
+def call_fc1(lib, **kw):
+    args = dict(X=FAKE, A=FAKE, a=FAKE, T=64, h=256, f=1024, t=2, Z=FAKE, H=FAKE, ws=FAKE * 2,
+                ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return lib.mlp_tp_fc1_forward(args["X"], args["A"], args["a"], args["T"], args["h"], args["f"], args["t"],
+                                  args["Z"], args["H"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(X=None), 1, "X is NULL"),
+    (dict(H=None), 1, "H is NULL"),
+    (dict(t=0), 1, "t=0"),
+    (dict(T=-5), 1, "negative"),
+    (dict(h=96), 2, "h=96"),
+    (dict(f=1025), 2, "not divisible"),
+    (dict(f=1024 + 64, t=2), 2, "multiple of 64"),
+    (dict(A=FAKE + 8), 3, "A is not 16-byte aligned"),
+    (dict(ws=None), 1, "workspace pointer is NULL"),
+    (dict(ws=FAKE + 16), 3, "workspace is not 256-byte aligned"),
+    (dict(ws_bytes=100), 4, "needs"),
+])
+def test_bad_arguments_are_rejected_on_the_host(lib, kw, status, needle):
+    st = call_fc1(lib, **kw)
+    assert st == status, binding.mlp_tp_last_error()
+    assert needle in binding.mlp_tp_last_error()
+
+
+def test_valid_arguments_without_a_gpu_report_the_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call_fc1(lib) == 5  # MLP_ERR_UNSUPPORTED_DEVICE, nothing launched
+
+
+def test_launch_counter_and_hooks_callable(lib):
+    c0 = binding.mlp_tp_launch_count()
+    binding.mlp_tp_set_wait_budget_ns(10)       # raised to the 1 ms floor
+    binding.mlp_tp_set_wait_budget_ns(1_000_000_000)
+    binding.mlp_tp_set_debug_flags(0)
+    assert binding.mlp_tp_launch_count() == c0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(64, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.mlp_tp_fc1_forward(x, x, x, 64, 256, 1024, 2, x, x, (FAKE, 1 << 30), stream=0)
