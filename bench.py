@@ -47,11 +47,14 @@ STAGES = ("fc1_forward", "fc2_forward", "fc2_backward_data", "fc2_backward_weigh
 STAGE_KERNEL = {
     "fc1_forward": "Z=X·A+a, H=GeLU(Z) (column-parallel GEMM, bias+GeLU epilogue)",
     "fc2_forward": "Y=Σ_i H_i·B_i + b (row-parallel GEMM, shard-sum epilogue)",
-    "fc2_backward_data": "dH=(dY·Bᵀ)⊙GeLU'(Z) (GEMM, GeLU-derivative epilogue)",
-    "fc2_backward_weight": "dB=Hᵀ·dY (GEMM) + db column sum",
+    "fc2_backward_data": "dH=(dY·Bᵀ)⊙GeLU'(Z), da (GEMM, GeLU-derivative + column-sum epilogue) + da reduce",
+    "fc2_backward_weight": "dB=(H+H_lo)ᵀ·dY (GEMM over both halves) + db column sum",
     "fc1_backward_data": "dX=Σ_i dH_i·A_iᵀ (GEMM, shard-sum epilogue)",
-    "fc1_backward_weight": "dA=Xᵀ·dH (GEMM) + da column sum",
+    "fc1_backward_weight": "dA=Xᵀ·(dH+dH_lo) (GEMM over both halves)",
 }
+# tensor-core products each stage's GEMM runs, in units of 2·T·h·f
+STAGE_PRODUCTS = {"fc1_forward": 1, "fc2_forward": 1, "fc2_backward_data": 1, "fc2_backward_weight": 2,
+                  "fc1_backward_data": 1, "fc1_backward_weight": 2}
 
 
 # ---------------------------------------------------------------- helpers
@@ -221,6 +224,8 @@ def main():
     ap.add_argument("--workload", default="h4096")
     ap.add_argument("--t", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--split", type=int, default=0,
+                    help="split flags: 1 = Y from the (H, H_lo) pair, 2 = dX from the (dH, dH_lo) pair")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -250,20 +255,24 @@ def main():
     host = inputs.make_inputs(wl, seed=wl.seed + rank)
     dev = {k: v.cuda() for k, v in host.items()}
     e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
-    Z, H, Y, dH = e(T, f), e(T, f), e(T, h), e(T, f)
+    Z = torch.empty(T, f, dtype=torch.float32, device="cuda")
+    H, H_lo, Y, dH, dH_lo = e(T, f), e(T, f), e(T, h), e(T, f), e(T, f)
     dX, dA, dB, da, db = e(T, h), e(h, f), e(f, h), e(f), e(h)
+    split = args.split
+    H_lo2 = H_lo if split & 1 else None
+    dH_lo2 = dH_lo if split & 2 else None
     ws = binding.make_workspace(T, h, f, t)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
     def step(evs=None):
         calls = (
-            lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, ws, sh),
-            lambda: binding.mlp_tp_fc2_forward(H, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
-            lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, ws, sh),
-            lambda: binding.mlp_tp_fc2_backward_weight(H, dev["dY"], T, h, f, t, dB, db, ws, sh),
-            lambda: binding.mlp_tp_fc1_backward_data(dH, dev["A"], T, h, f, t, dX, ws, sh),
-            lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], dH, T, h, f, t, dA, da, ws, sh),
+            lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, H_lo, ws, sh),
+            lambda: binding.mlp_tp_fc2_forward(H, H_lo2, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, dH_lo, da, ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t, dB, db, ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_data(dH, dH_lo2, dev["A"], T, h, f, t, dX, ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t, dA, ws, sh),
         )
         for i, c in enumerate(calls):
             if evs is not None:
@@ -315,8 +324,9 @@ def main():
     def e2e_step():
         for k, v in pin.items():
             dev[k].copy_(v, non_blocking=True)
-        binding.mlp_tp_forward(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, Y, Z, H, ws, sh)
-        binding.mlp_tp_backward(dev["dY"], dev["X"], dev["A"], dev["B"], Z, H, T, h, f, t,
+        binding.mlp_tp_forward(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, split,
+                               Y, Z, H, H_lo, ws, sh)
+        binding.mlp_tp_backward(dev["dY"], dev["X"], dev["A"], dev["B"], Z, H, H_lo, T, h, f, t, split,
                                 dX, dA, da, dB, db, ws, sh)
         for k, v in outs_host.items():
             v.copy_(outs_dev[k], non_blocking=True)
@@ -343,7 +353,10 @@ def main():
     # ------------------------------------------------ roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     dom = max(STAGES, key=lambda s: stage_ms[s])
-    gemm_flops = 2.0 * T * h * f
+    products = dict(STAGE_PRODUCTS)
+    products["fc2_forward"] += 1 if split & 1 else 0
+    products["fc1_backward_data"] += 1 if split & 2 else 0
+    gemm_flops = 2.0 * T * h * f * products[dom]
     achieved = gemm_flops / (stage_ms[dom] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     roofline = {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved,
@@ -356,7 +369,8 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, bf16)",
-        "config": workload_config(wl, t, world),
+        "config": dict(workload_config(wl, t, world), precision=precision_note(split),
+                       tensor_flops_per_step=2.0 * T * h * f * sum(products.values())),
         "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_DENSE_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * value / world / float(peaks.get("bf16_tflops", 1713.1)),
         "stage_ms": stage_ms,
@@ -370,6 +384,13 @@ def main():
         line["cpu_baseline"] = cpu_baseline(host, wl)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def precision_note(split):
+    y = "(H, H_lo) pair" if split & 1 else "bf16 H"
+    dx = "(dH, dH_lo) pair" if split & 2 else "bf16 dH"
+    return (f"bf16 inputs, fp32 accumulation; Z saved fp32; Y from {y}; dX from {dx}; dA, dB from the "
+            f"(hi, lo) bf16 pairs; da from fp32 dH")
 
 
 def traffic_for(stage, wl, t):

@@ -20,21 +20,33 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - All matrices are row-major, contiguous, bf16 (IEEE bfloat16), in device
- *    memory owned by the caller: X[T,h], A[h,f], a[f], B[f,h], b[h],
- *    Z[T,f], H[T,f], Y[T,h], dY[T,h], dH[T,f], dX[T,h], dA[h,f], da[f],
- *    dB[f,h], db[h].  Shard i owns columns [i·f/t, (i+1)·f/t) of A, a, Z, H,
- *    dH, dA, da and rows [i·f/t, (i+1)·f/t) of B and dB.
+ *  - All matrices are row-major and contiguous in device memory owned by the
+ *    caller.  bf16 (IEEE bfloat16): X[T,h], A[h,f], a[f], B[f,h], b[h],
+ *    Y[T,h], dY[T,h], dX[T,h], dA[h,f], da[f], dB[f,h], db[h], and the
+ *    pairs H, H_lo[T,f] and dH, dH_lo[T,f].  fp32: Z[T,f].  Shard i owns
+ *    columns [i·f/t, (i+1)·f/t) of A, a, Z, H, dH, dA, da and rows
+ *    [i·f/t, (i+1)·f/t) of B and dB.
+ *  - Saved activations.  The forward saves the pre-activation Z = X·A + a in
+ *    fp32 and the activation H = g(Z) as a bf16 pair (H, H_lo) with
+ *    H = bf16(g(Z)) and H_lo = bf16(g(Z) − H), about 16 significant bits.
+ *    The backward forms dH = (dY·Bᵀ) ⊙ g'(Z) in fp32 and keeps it as the
+ *    same kind of pair.  The weight gradients dA = Xᵀ·dH and dB = Hᵀ·dY
+ *    always use both halves of the pair (two bf16 tensor-core products);
+ *    Y and dX use only the high half unless the split flags below ask for
+ *    both.  da is summed from the fp32 dH before rounding.  With bf16-rounded
+ *    intermediates alone, the gradients of a unit-scale batch of a few
+ *    thousand tokens already differ from the exact block by more than
+ *    1e-2·(|exact| + 1); the pairs keep them well inside it.
  *  - Every device pointer must be 16-byte aligned.  Inputs are only read;
  *    outputs are overwritten (never accumulated into).  Outputs must not
  *    alias inputs or each other.
  *  - Shapes: T >= 0, h >= 64 and h % 64 == 0, t >= 1, f % t == 0,
  *    fs = f/t >= 64 and fs % 64 == 0, and T, h, f < 2^31.
  *  - `ws` is a caller-owned device workspace of at least
- *    mlp_tp_workspace_bytes(T, h, f, t) bytes, zero-filled once before its
- *    first use; the library keeps a device status word in its first bytes
- *    and scratch after it.  Calls that share a workspace must be ordered on
- *    one stream.
+ *    mlp_tp_workspace_bytes(T, h, f, t) bytes, 256-byte aligned and
+ *    zero-filled once before its first use; the library keeps a device
+ *    status word in its first bytes and scratch after it.  Calls that share
+ *    a workspace must be ordered on one stream.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point except mlp_tp_check synchronises, and
  *    none allocates or frees memory.
@@ -67,79 +79,93 @@ typedef enum {
 } mlp_status_t;
 
 /* Bytes of workspace needed by every entry point below for this shape
- * (the maximum over all of them): a 256-byte status header, the dH buffer
+ * (the maximum over all of them): a 256-byte status header, the dH pair
  * used by mlp_tp_backward, and fp32 column-sum partials.  Returns 0 for an
  * invalid shape. */
 size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
 
+/* Split flags of the composite calls: which second-layer products also use
+ * the low half of the activation pair.  The weight gradients always do. */
+typedef enum {
+  MLP_TP_SPLIT_NONE = 0,
+  MLP_TP_SPLIT_FC2_FORWARD = 1,       /* Y  = Σ_i (H_i + H_lo_i)·B_i + b    */
+  MLP_TP_SPLIT_FC1_BACKWARD_DATA = 2, /* dX = Σ_i (dH_i + dH_lo_i)·A_iᵀ     */
+  MLP_TP_SPLIT_ALL = 3
+} mlp_tp_split_t;
+
 /* ---------------------------------------------------------------- forward */
 
-/* Whole forward: mlp_tp_fc1_forward then mlp_tp_fc2_forward.
- * Writes Y[T,h] and saves Z[T,f] = X·A + a and H[T,f] = g(Z) for the
- * backward. */
+/* Whole forward: mlp_tp_fc1_forward then mlp_tp_fc2_forward (the latter
+ * given H_lo when `split` has MLP_TP_SPLIT_FC2_FORWARD).  Writes Y[T,h] and
+ * saves Z[T,f] (fp32), H[T,f] and H_lo[T,f] for the backward. */
 mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a,
                             const void* B, const void* b,
-                            int64_t T, int64_t h, int64_t f, int32_t t,
-                            void* Y, void* Z, void* H,
+                            int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                            void* Y, void* Z, void* H, void* H_lo,
                             void* ws, size_t ws_bytes, void* stream);
 
-/* ColumnParallelLinear of every shard plus the activation:
- * Z_i = X·A_i + a_i and H_i = g(Z_i), for all i in one launch (shard i is
- * the column block i of Z and H).  No reduction: the column split needs
- * none. */
+/* ColumnParallelLinear of every shard plus the activation, one launch:
+ * Z_i = X·A_i + a_i (fp32) and H_i = g(Z_i) as the pair (H_i, H_lo_i)
+ * (shard i is column block i of Z, H and H_lo).  No reduction: the column
+ * split needs none. */
 mlp_status_t mlp_tp_fc1_forward(const void* X, const void* A, const void* a,
                                 int64_t T, int64_t h, int64_t f, int32_t t,
-                                void* Z, void* H,
+                                void* Z, void* H, void* H_lo,
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* RowParallelLinear of every shard plus the reduce that stands in for the
- * forward all-reduce: P_i = H_i·B_i in fp32, Y = (((P_0 + P_1) + ...) +
- * P_{t-1}) + b, rounded once to bf16.  `b` may be NULL (no bias). */
-mlp_status_t mlp_tp_fc2_forward(const void* H, const void* B, const void* b,
+ * forward all-reduce: P_i = H_i·B_i (+ H_lo_i·B_i when H_lo is not NULL) in
+ * fp32, Y = (((P_0 + P_1) + ...) + P_{t-1}) + b, rounded once to bf16.
+ * `b` may be NULL (no bias); `H_lo` may be NULL (high half only). */
+mlp_status_t mlp_tp_fc2_forward(const void* H, const void* H_lo, const void* B, const void* b,
                                 int64_t T, int64_t h, int64_t f, int32_t t,
                                 void* Y,
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------- backward */
 
-/* Whole backward, given dY and the Z, H saved by the forward:
- * mlp_tp_fc2_backward_data (dH into the workspace), mlp_tp_fc2_backward_weight,
- * mlp_tp_fc1_backward_data and mlp_tp_fc1_backward_weight.
+/* Whole backward, given dY and Z, H, H_lo saved by the forward:
+ * mlp_tp_fc2_backward_data (dH pair into the workspace),
+ * mlp_tp_fc2_backward_weight, mlp_tp_fc1_backward_data (given dH_lo when
+ * `split` has MLP_TP_SPLIT_FC1_BACKWARD_DATA) and mlp_tp_fc1_backward_weight.
  * `da` and `db` may be NULL (bias gradients not wanted). */
 mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A,
-                             const void* B, const void* Z, const void* H,
-                             int64_t T, int64_t h, int64_t f, int32_t t,
+                             const void* B, const void* Z, const void* H, const void* H_lo,
+                             int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
                              void* dX, void* dA, void* da, void* dB, void* db,
                              void* ws, size_t ws_bytes, void* stream);
 
 /* Backward of the row-parallel layer through the activation, per shard:
- * dH_i = (dY·B_iᵀ) ⊙ g'(Z_i).  dY reaches every shard unchanged (the
- * reduce's backward is the identity).  Writes dH[T,f]. */
+ * dH_i = (dY·B_iᵀ) ⊙ g'(Z_i) in fp32, written as the pair (dH, dH_lo), and
+ * da = sum over rows of the fp32 dH (NULL: skip).  dY reaches every shard
+ * unchanged (the reduce's backward is the identity). */
 mlp_status_t mlp_tp_fc2_backward_data(const void* dY, const void* B, const void* Z,
                                       int64_t T, int64_t h, int64_t f, int32_t t,
-                                      void* dH,
+                                      void* dH, void* dH_lo, void* da,
                                       void* ws, size_t ws_bytes, void* stream);
 
-/* Weight gradients of the row-parallel layer: dB_i = H_iᵀ·dY (each shard's
- * own rows of dB, no reduction) and db = sum over rows of dY (NULL: skip). */
-mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* dY,
+/* Weight gradients of the row-parallel layer: dB_i = (H_i + H_lo_i)ᵀ·dY
+ * (each shard's own rows of dB, no reduction) and db = sum over rows of dY
+ * (NULL: skip). */
+mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* H_lo, const void* dY,
                                         int64_t T, int64_t h, int64_t f, int32_t t,
                                         void* dB, void* db,
                                         void* ws, size_t ws_bytes, void* stream);
 
 /* Input gradient of the column-parallel layer plus the reduce that stands in
- * for the copy operator's backward all-reduce: Q_i = dH_i·A_iᵀ in fp32,
- * dX = ((Q_0 + Q_1) + ...) + Q_{t-1}, rounded once to bf16. */
-mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* A,
+ * for the copy operator's backward all-reduce: Q_i = dH_i·A_iᵀ (+ dH_lo_i·A_iᵀ
+ * when dH_lo is not NULL) in fp32, dX = ((Q_0 + Q_1) + ...) + Q_{t-1},
+ * rounded once to bf16. */
+mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* dH_lo, const void* A,
                                       int64_t T, int64_t h, int64_t f, int32_t t,
                                       void* dX,
                                       void* ws, size_t ws_bytes, void* stream);
 
-/* Weight gradients of the column-parallel layer: dA_i = Xᵀ·dH_i (each
- * shard's own columns of dA) and da = sum over rows of dH (NULL: skip). */
-mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH,
+/* Weight gradient of the column-parallel layer: dA_i = Xᵀ·(dH_i + dH_lo_i)
+ * (each shard's own columns of dA, no reduction). */
+mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const void* dH_lo,
                                         int64_t T, int64_t h, int64_t f, int32_t t,
-                                        void* dA, void* da,
+                                        void* dA,
                                         void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------ diagnostics */

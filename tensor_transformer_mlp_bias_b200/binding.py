@@ -34,14 +34,14 @@ _I32 = ctypes.c_int32
 _SZ = ctypes.c_size_t
 _SIGS = {
     "mlp_tp_workspace_bytes": ([_I64, _I64, _I64, _I32], _SZ),
-    "mlp_tp_forward": ([_P] * 5 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc1_forward": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc2_forward": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_backward": ([_P] * 6 + [_I64, _I64, _I64, _I32] + [_P] * 5 + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc2_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc2_backward_weight": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc1_backward_data": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
-    "mlp_tp_fc1_backward_weight": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_forward": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 4 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_forward": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_forward": ([_P] * 4 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_backward": ([_P] * 7 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 5 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_check": ([_P, _P], ctypes.c_int),
     "mlp_tp_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "mlp_tp_last_error": ([], ctypes.c_char_p),
@@ -49,6 +49,12 @@ _SIGS = {
     "mlp_tp_set_wait_budget_ns": ([ctypes.c_uint64], None),
     "mlp_tp_set_debug_flags": ([ctypes.c_uint32], None),
 }
+
+# split flags of the composite calls (mlp_tp_split_t)
+SPLIT_NONE = 0
+SPLIT_FC2_FORWARD = 1
+SPLIT_FC1_BACKWARD_DATA = 2
+SPLIT_ALL = 3
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -93,8 +99,9 @@ def _addr(x, name: str, nullable: bool = False):
         raise TypeError(f"{name}: expected a torch.Tensor or an int address")
     if x.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor (got {x.device})")
-    if x.dtype != torch.bfloat16 and name != "ws":
-        raise ValueError(f"{name} must be bfloat16 (got {x.dtype})")
+    want = torch.float32 if name == "Z" else torch.bfloat16
+    if name != "ws" and x.dtype != want:
+        raise ValueError(f"{name} must be {want} (got {x.dtype})")
     if not x.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return x.data_ptr()
@@ -136,54 +143,56 @@ def make_workspace(T: int, h: int, f: int, t: int, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def mlp_tp_forward(X, A, a, B, b, T, h, f, t, Y, Z, H, ws, stream=None):
+def mlp_tp_forward(X, A, a, B, b, T, h, f, t, split, Y, Z, H, H_lo, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"), _addr(b, "b"),
-                                T, h, f, t, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"), w, wn, _stream(stream)))
+                                T, h, f, t, split, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"),
+                                _addr(H_lo, "H_lo"), w, wn, _stream(stream)))
 
 
-def mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, ws, stream=None):
+def mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, H_lo, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_fc1_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), T, h, f, t,
-                                    _addr(Z, "Z"), _addr(H, "H"), w, wn, _stream(stream)))
+                                    _addr(Z, "Z"), _addr(H, "H"), _addr(H_lo, "H_lo"), w, wn, _stream(stream)))
 
 
-def mlp_tp_fc2_forward(H, B, b, T, h, f, t, Y, ws, stream=None):
+def mlp_tp_fc2_forward(H, H_lo, B, b, T, h, f, t, Y, ws, stream=None):
     w, wn = _ws(ws)
-    _check(lib().mlp_tp_fc2_forward(_addr(H, "H"), _addr(B, "B"), _addr(b, "b", True), T, h, f, t,
-                                    _addr(Y, "Y"), w, wn, _stream(stream)))
+    _check(lib().mlp_tp_fc2_forward(_addr(H, "H"), _addr(H_lo, "H_lo", True), _addr(B, "B"), _addr(b, "b", True),
+                                    T, h, f, t, _addr(Y, "Y"), w, wn, _stream(stream)))
 
 
-def mlp_tp_backward(dY, X, A, B, Z, H, T, h, f, t, dX, dA, da, dB, db, ws, stream=None):
+def mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, split, dX, dA, da, dB, db, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_backward(_addr(dY, "dY"), _addr(X, "X"), _addr(A, "A"), _addr(B, "B"), _addr(Z, "Z"),
-                                 _addr(H, "H"), T, h, f, t, _addr(dX, "dX"), _addr(dA, "dA"),
-                                 _addr(da, "da", True), _addr(dB, "dB"), _addr(db, "db", True), w, wn,
-                                 _stream(stream)))
+                                 _addr(H, "H"), _addr(H_lo, "H_lo"), T, h, f, t, split, _addr(dX, "dX"),
+                                 _addr(dA, "dA"), _addr(da, "da", True), _addr(dB, "dB"), _addr(db, "db", True),
+                                 w, wn, _stream(stream)))
 
 
-def mlp_tp_fc2_backward_data(dY, B, Z, T, h, f, t, dH, ws, stream=None):
+def mlp_tp_fc2_backward_data(dY, B, Z, T, h, f, t, dH, dH_lo, da, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_fc2_backward_data(_addr(dY, "dY"), _addr(B, "B"), _addr(Z, "Z"), T, h, f, t,
-                                          _addr(dH, "dH"), w, wn, _stream(stream)))
-
-
-def mlp_tp_fc2_backward_weight(H, dY, T, h, f, t, dB, db, ws, stream=None):
-    w, wn = _ws(ws)
-    _check(lib().mlp_tp_fc2_backward_weight(_addr(H, "H"), _addr(dY, "dY"), T, h, f, t, _addr(dB, "dB"),
-                                            _addr(db, "db", True), w, wn, _stream(stream)))
-
-
-def mlp_tp_fc1_backward_data(dH, A, T, h, f, t, dX, ws, stream=None):
-    w, wn = _ws(ws)
-    _check(lib().mlp_tp_fc1_backward_data(_addr(dH, "dH"), _addr(A, "A"), T, h, f, t, _addr(dX, "dX"),
+                                          _addr(dH, "dH"), _addr(dH_lo, "dH_lo"), _addr(da, "da", True),
                                           w, wn, _stream(stream)))
 
 
-def mlp_tp_fc1_backward_weight(X, dH, T, h, f, t, dA, da, ws, stream=None):
+def mlp_tp_fc2_backward_weight(H, H_lo, dY, T, h, f, t, dB, db, ws, stream=None):
     w, wn = _ws(ws)
-    _check(lib().mlp_tp_fc1_backward_weight(_addr(X, "X"), _addr(dH, "dH"), T, h, f, t, _addr(dA, "dA"),
-                                            _addr(da, "da", True), w, wn, _stream(stream)))
+    _check(lib().mlp_tp_fc2_backward_weight(_addr(H, "H"), _addr(H_lo, "H_lo"), _addr(dY, "dY"), T, h, f, t,
+                                            _addr(dB, "dB"), _addr(db, "db", True), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_data(dH, dH_lo, A, T, h, f, t, dX, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_data(_addr(dH, "dH"), _addr(dH_lo, "dH_lo", True), _addr(A, "A"),
+                                          T, h, f, t, _addr(dX, "dX"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_weight(X, dH, dH_lo, T, h, f, t, dA, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_weight(_addr(X, "X"), _addr(dH, "dH"), _addr(dH_lo, "dH_lo"), T, h, f, t,
+                                            _addr(dA, "dA"), w, wn, _stream(stream)))
 
 
 def mlp_tp_check(ws, stream=None):

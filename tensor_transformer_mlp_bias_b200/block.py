@@ -12,7 +12,8 @@ from . import binding
 
 def alloc_outputs(T: int, h: int, f: int, device="cuda", with_bias_grads: bool = True) -> Dict[str, torch.Tensor]:
     e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device=device)  # noqa: E731
-    out = {"Y": e(T, h), "Z": e(T, f), "H": e(T, f), "dX": e(T, h), "dA": e(h, f), "dB": e(f, h)}
+    out = {"Y": e(T, h), "Z": torch.empty(T, f, dtype=torch.float32, device=device), "H": e(T, f),
+           "H_lo": e(T, f), "dX": e(T, h), "dA": e(h, f), "dB": e(f, h)}
     if with_bias_grads:
         out["da"] = e(f)
         out["db"] = e(h)
@@ -20,23 +21,25 @@ def alloc_outputs(T: int, h: int, f: int, device="cuda", with_bias_grads: bool =
 
 
 def forward(inp: Dict[str, torch.Tensor], t: int, out: Dict[str, torch.Tensor], ws: torch.Tensor,
-            stream=None) -> None:
+            split: int = binding.SPLIT_NONE, stream=None) -> None:
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
-    binding.mlp_tp_forward(inp["X"], inp["A"], inp["a"], inp["B"], inp["b"], T, h, f, t,
-                           out["Y"], out["Z"], out["H"], ws, stream)
+    binding.mlp_tp_forward(inp["X"], inp["A"], inp["a"], inp["B"], inp["b"], T, h, f, t, split,
+                           out["Y"], out["Z"], out["H"], out["H_lo"], ws, stream)
 
 
 def backward(inp: Dict[str, torch.Tensor], t: int, out: Dict[str, torch.Tensor], ws: torch.Tensor,
-             stream=None) -> None:
+             split: int = binding.SPLIT_NONE, stream=None) -> None:
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
-    binding.mlp_tp_backward(inp["dY"], inp["X"], inp["A"], inp["B"], out["Z"], out["H"], T, h, f, t,
-                            out["dX"], out["dA"], out.get("da"), out["dB"], out.get("db"), ws, stream)
+    binding.mlp_tp_backward(inp["dY"], inp["X"], inp["A"], inp["B"], out["Z"], out["H"], out["H_lo"],
+                            T, h, f, t, split, out["dX"], out["dA"], out.get("da"), out["dB"], out.get("db"),
+                            ws, stream)
 
 
 def forward_backward(inp: Dict[str, torch.Tensor], t: int, out: Optional[Dict[str, torch.Tensor]] = None,
-                     ws: Optional[torch.Tensor] = None, check: bool = True) -> Dict[str, torch.Tensor]:
+                     ws: Optional[torch.Tensor] = None, split: int = binding.SPLIT_NONE,
+                     check: bool = True) -> Dict[str, torch.Tensor]:
     """Run forward then backward on the current stream; returns the outputs."""
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
@@ -45,8 +48,8 @@ def forward_backward(inp: Dict[str, torch.Tensor], t: int, out: Optional[Dict[st
         out = alloc_outputs(T, h, f, dev)
     if ws is None:
         ws = binding.make_workspace(T, h, f, t, dev)
-    forward(inp, t, out, ws)
-    backward(inp, t, out, ws)
+    forward(inp, t, out, ws, split)
+    backward(inp, t, out, ws, split)
     if check:
         binding.mlp_tp_check(ws)
     return out

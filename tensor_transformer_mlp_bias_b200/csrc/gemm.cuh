@@ -13,8 +13,8 @@
 //               barrier and each finished accumulator to a "tmem full"
 //               barrier;
 //   warps 2-9   epilogue: tcgen05.ld the accumulator (one row per thread,
-//               32 columns per load), apply the fused math, store bf16 to
-//               global memory, release the accumulator.
+//               32 columns per load), apply the fused math, store to global
+//               memory, release the accumulator.
 // The two accumulators let the epilogue of one unit overlap the mainloop of
 // the next.
 //
@@ -25,6 +25,12 @@
 // epilogue receives the t shard partials P_0..P_{t-1} separately and sums
 // them in registers in ascending shard order, adds the bias and rounds once.
 // This is the on-device stand-in for the tensor-parallel all-reduce.
+//
+// Split operands.  An activation or gradient that is computed here (H, dH)
+// is kept as a bf16 pair v = hi + lo (hi = bf16(v), lo = bf16(v - hi), about
+// 16 significant bits).  A product that must see that precision runs its K
+// loop twice ("parts"): once over (hi, other operand) and once over
+// (lo, other operand), accumulating into the same TMEM accumulator.
 //
 // Operand layouts.  A K-major operand is stored [rows, K] with K contiguous
 // and arrives as one TMA box of 64 (K) x rows.  An MN-major operand is
@@ -67,15 +73,25 @@ enum Epi : int { EPI_BIAS_GELU = 0, EPI_SHARD_SUM = 1, EPI_GELU_GRAD = 2, EPI_ST
 struct GemmParams {
   int M, N;
   int shards;             // K segments reduced in the epilogue (EPI_SHARD_SUM); 1 otherwise
-  int kblocks_per_shard;  // BK-wide K slices per segment
+  int parts;              // 1, or 2 when an operand is a bf16 (hi, lo) pair
+  int kblocks_per_shard;  // BK-wide K slices per segment and part
   int m_blocks, n_blocks, num_tiles, group_m;
-  __nv_bfloat16* out0;        // Z | Y | dH | dX | dA | dB
-  __nv_bfloat16* out1;        // H (EPI_BIAS_GELU)
+  __nv_bfloat16* out0;        // H_hi | Y | dH_hi | dX | dA | dB
+  __nv_bfloat16* out1;        // H_lo (EPI_BIAS_GELU) | dH_lo (EPI_GELU_GRAD)
+  float* out_f32;             // Z (EPI_BIAS_GELU)
+  float* colsum;              // [m_blocks*4, N] column sums of dH (EPI_GELU_GRAD), may be null
   const __nv_bfloat16* bias;  // a (EPI_BIAS_GELU) or b (EPI_SHARD_SUM), may be null for the latter
-  const __nv_bfloat16* aux;   // Z (EPI_GELU_GRAD)
+  const float* aux;           // Z (EPI_GELU_GRAD)
   unsigned int* status;       // device status word pair in the workspace
   unsigned long long budget_ns;
   unsigned int debug_flags;
+};
+
+// Tensor maps of the operands, one per K part (part 1 repeats part 0 for an
+// operand that is not split).
+struct GemmMaps {
+  CUtensorMap a[2];
+  CUtensorMap b[2];
 };
 
 struct GemmCtl {
@@ -156,6 +172,13 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
   return __bfloat1622float2(b);
 }
 
+// v0, v1 -> (hi pair, lo pair): hi = bf16(v), lo = bf16(v - hi).
+__device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(v0, v1);
+  const float2 h = unpack_bf16x2(hi);
+  lo = pack_bf16x2(v0 - h.x, v1 - h.y);
+}
+
 // 32 consecutive bf16 values -> fp32 (vectorised 16-byte loads).
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&dst)[32]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
@@ -172,6 +195,18 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&d
   }
 }
 
+__device__ __forceinline__ void load_f32x32(const float* src, float (&dst)[32]) {
+  const float4* s = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const float4 w = __ldg(s + v);
+    dst[4 * v] = w.x;
+    dst[4 * v + 1] = w.y;
+    dst[4 * v + 2] = w.z;
+    dst[4 * v + 3] = w.w;
+  }
+}
+
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -179,11 +214,37 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
     d[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
 }
 
+__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+// Column sums over the warp's 32 rows: lane r holds row r's 32 values; on
+// return lane j holds the sum over rows of column j.  Recursive halving:
+// at each step a lane keeps the half of its columns selected by one bit of
+// its lane index and adds the partner lane's copy of that half (31 shuffles
+// in all, fixed order, so the result is deterministic).
+__device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int half = 16 >> step;           // values kept after this step
+    const bool upper = (lane & half) != 0;  // keep the upper half of the current columns
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float send = upper ? v[j] : v[j + half];
+      const float keep = upper ? v[j + half] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
 // ---------------------------------------------------------------- kernel
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    mlp_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                    const GemmParams p) {
+    mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -210,8 +271,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tma_a);
-    prefetch_tensormap(&tma_b);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      prefetch_tensormap(&maps.a[i]);
+      prefetch_tensormap(&maps.b[i]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -223,7 +287,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
   const uint64_t budget = p.budget_ns;
-  const int total_kb = p.shards * p.kblocks_per_shard;
+  const int kb_per_unit = p.parts * p.kblocks_per_shard;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -232,42 +296,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage: filled at least once / parity of last fill
       bool ok = true;
+      bool first = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         int mb, nb;
         tile_coords(tile, p, mb, nb);
         const int m0 = mb * BM, n0 = nb * BN;
-        for (int kb = 0; kb < total_kb; ++kb) {
-          if ((p.debug_flags & 1u) && (tile != (int)blockIdx.x || kb >= 1)) {
-            ok = false;  // test hook: stop feeding the tensor core
-            break;
-          }
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, budget)) {
-            record_timeout(p, abort_flag, 0x100u);
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(&ctl->full[stage]);
-          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
-          const int k0 = kb * BK;
-          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
-          if (A_MN) {
-            tma_load_2d(a_dst, &tma_a, fb, m0, k0);
-            tma_load_2d(a_dst + MN_BOX_BYTES, &tma_a, fb, m0 + 64, k0);
-          } else {
-            tma_load_2d(a_dst, &tma_a, fb, k0, m0);
-          }
-          if (B_MN) {
+        for (int s = 0; ok && s < p.shards; ++s) {
+          for (int i = 0; i < kb_per_unit; ++i) {
+            if ((p.debug_flags & 1u) && !first) {
+              ok = false;  // test hook: stop feeding the tensor core after one stage
+              break;
+            }
+            first = false;
+            if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag, budget)) {
+              record_timeout(p, abort_flag, 0x100u);
+              ok = false;
+              break;
+            }
+            const int part = i / p.kblocks_per_shard;
+            const int k0 = (s * p.kblocks_per_shard + (i - part * p.kblocks_per_shard)) * BK;
+            const CUtensorMap* ma = &maps.a[part];
+            const CUtensorMap* mbp = &maps.b[part];
+            const uint32_t fb = smem_u32(&ctl->full[stage]);
+            mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
+            const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
+            const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
+            if (A_MN) {
+              tma_load_2d(a_dst, ma, fb, m0, k0);
+              tma_load_2d(a_dst + MN_BOX_BYTES, ma, fb, m0 + 64, k0);
+            } else {
+              tma_load_2d(a_dst, ma, fb, k0, m0);
+            }
+            if (B_MN) {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * MN_BOX_BYTES, &tma_b, fb, n0 + 64 * j, k0);
-          } else {
-            tma_load_2d(b_dst, &tma_b, fb, k0, n0);
-          }
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
+            } else {
+              tma_load_2d(b_dst, mbp, fb, k0, n0);
+            }
+            issued_mask |= 1u << stage;
+            issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
@@ -294,7 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after_sync();
           const uint32_t d_tmem = tmem_base + acc * BN;
-          for (int kb = 0; kb < p.kblocks_per_shard; ++kb) {
+          for (int i = 0; i < kb_per_unit; ++i) {
             if (!mbar_wait(&ctl->full[stage], phase, abort_flag, budget)) {
               record_timeout(p, abort_flag, 0x300u);
               ok = false;
@@ -313,7 +384,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
               const uint64_t bd = B_MN ? smem_desc_sw128(b_base + k * 2048, MN_BOX_BYTES, 1024)
                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
-              mma_bf16_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+              mma_bf16_ss(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
             }
             mma_commit(&ctl->empty[stage]);
             if (++stage == STAGES) {
@@ -359,34 +430,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t r[32];
           tmem_load_32cols(t_addr + c * 32, r);
           if constexpr (EPI == EPI_BIAS_GELU) {
+            // Z = X·A + a (fp32, saved), H = g(Z) saved as (hi, lo)
             float bias[32];
             load_bf16x32(p.bias + col, bias);
-            uint32_t zp[16], hp[16];
+            float z[32];
+            uint32_t hp[16], lp[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float z0 = __uint_as_float(r[2 * j]) + bias[2 * j];
-              const float z1 = __uint_as_float(r[2 * j + 1]) + bias[2 * j + 1];
-              zp[j] = pack_bf16x2(z0, z1);
-              hp[j] = pack_bf16x2(gelu_f(z0), gelu_f(z1));
-            }
+            for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(r[j]) + bias[j];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) split_bf16x2(gelu_f(z[2 * j]), gelu_f(z[2 * j + 1]), hp[j], lp[j]);
             if (row_ok) {
-              store_bf16x32(p.out0 + row_off + col, zp);
-              store_bf16x32(p.out1 + row_off + col, hp);
+              store_f32x32(p.out_f32 + row_off + col, z);
+              store_bf16x32(p.out0 + row_off + col, hp);
+              store_bf16x32(p.out1 + row_off + col, lp);
             }
           } else if constexpr (EPI == EPI_GELU_GRAD) {
+            // dH = (dY·Bᵀ) ⊙ g'(Z), saved as (hi, lo); fp32 column sums for da
             float z[32];
             if (row_ok) {
-              load_bf16x32(p.aux + row_off + col, z);
+              load_f32x32(p.aux + row_off + col, z);
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j) z[j] = 0.0f;
             }
-            uint32_t dp[16];
+            float dh[32];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              dp[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * gelu_grad_f(z[2 * j]),
-                                  __uint_as_float(r[2 * j + 1]) * gelu_grad_f(z[2 * j + 1]));
-            if (row_ok) store_bf16x32(p.out0 + row_off + col, dp);
+            for (int j = 0; j < 32; ++j) dh[j] = row_ok ? __uint_as_float(r[j]) * gelu_grad_f(z[j]) : 0.0f;
+            uint32_t hp[16], lp[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) split_bf16x2(dh[2 * j], dh[2 * j + 1], hp[j], lp[j]);
+            if (row_ok) {
+              store_bf16x32(p.out0 + row_off + col, hp);
+              store_bf16x32(p.out1 + row_off + col, lp);
+            }
+            if (p.colsum != nullptr) {
+              const float cs = warp_column_sums(dh);
+              p.colsum[static_cast<size_t>(mb * 4 + q) * p.N + col + lane] = cs;
+            }
           } else if constexpr (EPI == EPI_STORE) {
             uint32_t op[16];
 #pragma unroll

@@ -66,24 +66,32 @@ mlp_status_t check_shape(const Shape& s) {
 }
 
 size_t colsum_chunks(int64_t R) { return static_cast<size_t>((R + COLSUM_ROWS_PER_CHUNK - 1) / COLSUM_ROWS_PER_CHUNK); }
+size_t gemm_row_blocks(int64_t R) { return static_cast<size_t>((R + BM - 1) / BM); }
 
+// Workspace layout: [status header | dH | dH_lo | fp32 column-sum partials].
+size_t pair_bytes(const Shape& s) { return align_up(static_cast<size_t>(s.T * s.f * 2), 256); }
 size_t dh_offset() { return WS_HEADER_BYTES; }
-size_t partial_offset(const Shape& s) { return WS_HEADER_BYTES + align_up(static_cast<size_t>(s.T * s.f * 2), 256); }
+size_t dh_lo_offset(const Shape& s) { return WS_HEADER_BYTES + pair_bytes(s); }
+size_t partial_offset(const Shape& s) { return WS_HEADER_BYTES + 2 * pair_bytes(s); }
 size_t workspace_bytes(const Shape& s) {
-  const size_t cols = static_cast<size_t>(s.f > s.h ? s.f : s.h);
-  return partial_offset(s) + align_up(colsum_chunks(s.T) * cols * sizeof(float), 256);
+  // da: one row of column sums per (128-row block, 32-row lane quadrant);
+  // db: one row per COLSUM_ROWS_PER_CHUNK rows of dY.
+  const size_t da_rows = gemm_row_blocks(s.T) * 4 * static_cast<size_t>(s.f);
+  const size_t db_rows = colsum_chunks(s.T) * static_cast<size_t>(s.h);
+  return partial_offset(s) + align_up((da_rows > db_rows ? da_rows : db_rows) * sizeof(float), 256);
 }
 
 struct Ptr {
   const void* p;
   const char* name;
   bool nullable;
+  bool empty = false;  // the buffer holds no elements (a T-sized buffer with T == 0): NULL is fine
 };
 
 mlp_status_t check_ptrs(std::initializer_list<Ptr> ptrs) {
   for (const Ptr& x : ptrs) {
     if (x.p == nullptr) {
-      if (x.nullable) continue;
+      if (x.nullable || x.empty) continue;
       return fail(MLP_ERR_INVALID_ARG, "pointer %s is NULL", x.name);
     }
     if (reinterpret_cast<uintptr_t>(x.p) % 16 != 0)
@@ -176,13 +184,16 @@ mlp_status_t make_operand_map(CUtensorMap* map, const void* ptr, bool mn_major, 
 }
 
 // ---------------------------------------------------------------- launches
+struct Operand {
+  const void* p[2];  // part 0 and part 1 (part 1 = part 0 when not split)
+  bool mn_major;
+};
+
 struct GemmDesc {
-  const void* a;  // Aop
-  bool a_mn;
-  const void* b;  // Bop
-  bool b_mn;
-  int64_t M, N, K;  // K = shards * kseg
+  Operand a, b;
+  int64_t M, N, K;  // K = shards * (K of one shard); each part spans all of K
   int shards;
+  int parts;
 };
 
 int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
@@ -193,18 +204,41 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
   return m_blocks < 16 ? m_blocks : 16;
 }
 
+// One opt-in per kernel instantiation and device (the static state is per
+// template instance).
 template <bool A_MN, bool B_MN, int EPI>
-mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, int sms, cudaStream_t stream, const char* name) {
-  if (g.M == 0 || g.N == 0) return MLP_OK;
-  CUtensorMap ma, mb;
-  mlp_status_t st = make_operand_map(&ma, g.a, A_MN, g.M, g.K, BM, name);
-  if (st != MLP_OK) return st;
-  st = make_operand_map(&mb, g.b, B_MN, g.N, g.K, BN, name);
-  if (st != MLP_OK) return st;
+mlp_status_t ensure_smem_attr(int dev) {
+  static std::mutex mu;
+  static uint64_t done_mask = 0;
+  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI>;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done_mask & (1ull << dev)) return MLP_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+  done_mask |= 1ull << dev;
+  return MLP_OK;
+}
 
+struct Launch {
+  int dev;
+  int sms;
+  cudaStream_t stream;
+};
+
+template <bool A_MN, bool B_MN, int EPI>
+mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
+  if (g.M == 0 || g.N == 0) return MLP_OK;
+  GemmMaps maps;
+  for (int i = 0; i < 2; ++i) {
+    mlp_status_t st = make_operand_map(&maps.a[i], g.a.p[i], A_MN, g.M, g.K, BM, name);
+    if (st != MLP_OK) return st;
+    st = make_operand_map(&maps.b[i], g.b.p[i], B_MN, g.N, g.K, BN, name);
+    if (st != MLP_OK) return st;
+  }
   p.M = static_cast<int>(g.M);
   p.N = static_cast<int>(g.N);
   p.shards = g.shards;
+  p.parts = g.parts;
   p.kblocks_per_shard = static_cast<int>((g.K / g.shards + BK - 1) / BK);
   p.m_blocks = static_cast<int>((g.M + BM - 1) / BM);
   p.n_blocks = static_cast<int>((g.N + BN - 1) / BN);
@@ -213,18 +247,21 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, int sms, cudaStream_t 
   p.budget_ns = g_budget_ns.load();
   p.debug_flags = g_debug_flags.load();
 
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(mlp_gemm_kernel<A_MN, B_MN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    GEMM_SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(max dynamic shared memory)");
-
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  mlp_gemm_kernel<A_MN, B_MN, EPI><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, stream>>>(ma, mb, p);
+  mlp_status_t st = ensure_smem_attr<A_MN, B_MN, EPI>(L.dev);
+  if (st != MLP_OK) return st;
+  const int grid = p.num_tiles < L.sms ? p.num_tiles : L.sms;
+  mlp_gemm_kernel<A_MN, B_MN, EPI><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, L.stream>>>(maps, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
+  g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+mlp_status_t launch_colsum_final(const float* partial, int chunks, int64_t C, void* out, cudaStream_t stream) {
+  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(partial, chunks, static_cast<int>(C),
+                                                                           static_cast<__nv_bfloat16*>(out));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "colsum_final");
   g_launches.fetch_add(1);
   return MLP_OK;
 }
@@ -241,12 +278,12 @@ mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "colsum_partial");
   g_launches.fetch_add(1);
-  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(partial, chunks, static_cast<int>(C),
-                                                                           static_cast<__nv_bfloat16*>(out));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "colsum_final");
-  g_launches.fetch_add(1);
-  return MLP_OK;
+  return launch_colsum_final(partial, chunks, C, out, stream);
+}
+
+mlp_status_t zero_fill(void* p, size_t bytes, cudaStream_t s, const char* what) {
+  cudaError_t e = cudaMemsetAsync(p, 0, bytes, s);
+  return e == cudaSuccess ? MLP_OK : cuda_fail(e, what);
 }
 
 GemmParams base_params(void* ws) {
@@ -256,87 +293,96 @@ GemmParams base_params(void* ws) {
   return p;
 }
 
-// ---------------------------------------------------------------- stages
-mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H, void* ws,
-                         int sms, cudaStream_t st) {
-  GemmParams p = base_params(ws);
-  p.out0 = static_cast<__nv_bfloat16*>(Z);
-  p.out1 = static_cast<__nv_bfloat16*>(H);
-  p.bias = static_cast<const __nv_bfloat16*>(a);
-  GemmDesc g{X, false, A, true, s.T, s.f, s.h, 1};
-  return launch_gemm<false, true, EPI_BIAS_GELU>(g, p, sms, st, "column-parallel forward (Z, H)");
+Operand one(const void* p, bool mn) { return Operand{{p, p}, mn}; }
+Operand pair(const void* hi, const void* lo, bool mn) { return Operand{{hi, lo != nullptr ? lo : hi}, mn}; }
+float* partials(void* ws, const Shape& s) {
+  return reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
 }
 
-mlp_status_t fc2_forward(const Shape& s, const void* H, const void* B, const void* b, void* Y, void* ws, int sms,
-                         cudaStream_t st) {
+// ---------------------------------------------------------------- stages
+mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H, void* H_lo,
+                         void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.out_f32 = static_cast<float*>(Z);
+  p.out0 = static_cast<__nv_bfloat16*>(H);
+  p.out1 = static_cast<__nv_bfloat16*>(H_lo);
+  p.bias = static_cast<const __nv_bfloat16*>(a);
+  GemmDesc g{one(X, false), one(A, true), s.T, s.f, s.h, 1, 1};
+  return launch_gemm<false, true, EPI_BIAS_GELU>(g, p, L, "column-parallel forward (Z, H)");
+}
+
+mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const void* B, const void* b, void* Y,
+                         void* ws, const Launch& L) {
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(Y);
   p.bias = static_cast<const __nv_bfloat16*>(b);
-  GemmDesc g{H, false, B, true, s.T, s.h, s.f, s.t};
-  return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, sms, st, "row-parallel forward + shard reduce (Y)");
+  GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, s.t, H_lo != nullptr ? 2 : 1};
+  return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, L, "row-parallel forward + shard reduce (Y)");
 }
 
-mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, const void* Z, void* dH, void* ws,
-                               int sms, cudaStream_t st) {
+mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, const void* Z, void* dH, void* dH_lo,
+                               void* da, void* ws, const Launch& L) {
+  if (s.T == 0) return da != nullptr ? zero_fill(da, static_cast<size_t>(s.f) * 2, L.stream, "cudaMemsetAsync(da)")
+                                     : MLP_OK;
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dH);
-  p.aux = static_cast<const __nv_bfloat16*>(Z);
-  GemmDesc g{dY, false, B, false, s.T, s.f, s.h, 1};
-  return launch_gemm<false, false, EPI_GELU_GRAD>(g, p, sms, st, "row-parallel backward data (dH)");
+  p.out1 = static_cast<__nv_bfloat16*>(dH_lo);
+  p.aux = static_cast<const float*>(Z);
+  p.colsum = da != nullptr ? partials(ws, s) : nullptr;
+  GemmDesc g{one(dY, false), one(B, false), s.T, s.f, s.h, 1, 1};
+  mlp_status_t st = launch_gemm<false, false, EPI_GELU_GRAD>(g, p, L, "row-parallel backward data (dH, da)");
+  if (st != MLP_OK || da == nullptr) return st;
+  return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream);
 }
 
-mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* dY, void* dB, void* db, void* ws,
-                                 int sms, cudaStream_t st) {
+mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* H_lo, const void* dY, void* dB, void* db,
+                                 void* ws, const Launch& L) {
+  mlp_status_t st;
   if (s.T == 0) {
-    cudaError_t e = cudaMemsetAsync(dB, 0, static_cast<size_t>(s.f * s.h * 2), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dB)");
+    st = zero_fill(dB, static_cast<size_t>(s.f * s.h * 2), L.stream, "cudaMemsetAsync(dB)");
   } else {
     GemmParams p = base_params(ws);
     p.out0 = static_cast<__nv_bfloat16*>(dB);
-    GemmDesc g{H, true, dY, true, s.f, s.h, s.T, 1};
-    mlp_status_t r = launch_gemm<true, true, EPI_STORE>(g, p, sms, st, "row-parallel weight gradient (dB)");
-    if (r != MLP_OK) return r;
+    GemmDesc g{pair(H, H_lo, true), one(dY, true), s.f, s.h, s.T, 1, 2};
+    st = launch_gemm<true, true, EPI_STORE>(g, p, L, "row-parallel weight gradient (dB)");
   }
-  if (db == nullptr) return MLP_OK;
-  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
-  return launch_colsum(dY, s.T, s.h, db, partial, st);
+  if (st != MLP_OK || db == nullptr) return st;
+  return launch_colsum(dY, s.T, s.h, db, partials(ws, s), L.stream);
 }
 
-mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* A, void* dX, void* ws, int sms,
-                               cudaStream_t st) {
+mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* dH_lo, const void* A, void* dX, void* ws,
+                               const Launch& L) {
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dX);
-  GemmDesc g{dH, false, A, false, s.T, s.h, s.f, s.t};
-  return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, sms, st, "column-parallel backward data + shard reduce (dX)");
+  GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, s.t, dH_lo != nullptr ? 2 : 1};
+  return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, L, "column-parallel backward data + shard reduce (dX)");
 }
 
-mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, void* dA, void* da, void* ws, int sms,
-                                 cudaStream_t st) {
-  if (s.T == 0) {
-    cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(s.h * s.f * 2), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dA)");
-  } else {
-    GemmParams p = base_params(ws);
-    p.out0 = static_cast<__nv_bfloat16*>(dA);
-    GemmDesc g{X, true, dH, true, s.h, s.f, s.T, 1};
-    mlp_status_t r = launch_gemm<true, true, EPI_STORE>(g, p, sms, st, "column-parallel weight gradient (dA)");
-    if (r != MLP_OK) return r;
-  }
-  if (da == nullptr) return MLP_OK;
-  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
-  return launch_colsum(dH, s.T, s.f, da, partial, st);
+mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, const void* dH_lo, void* dA, void* ws,
+                                 const Launch& L) {
+  if (s.T == 0) return zero_fill(dA, static_cast<size_t>(s.h * s.f * 2), L.stream, "cudaMemsetAsync(dA)");
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dA);
+  GemmDesc g{one(X, true), pair(dH, dH_lo, true), s.h, s.f, s.T, 1, 2};
+  return launch_gemm<true, true, EPI_STORE>(g, p, L, "column-parallel weight gradient (dA)");
 }
 
 // Common preamble: shape, pointers, workspace, device.
-mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, int& sms) {
+mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, void* stream,
+                      Launch& L) {
   mlp_status_t st = check_shape(s);
   if (st != MLP_OK) return st;
   st = check_ptrs(ptrs);
   if (st != MLP_OK) return st;
   st = check_ws(s, ws, ws_bytes);
   if (st != MLP_OK) return st;
-  int dev = 0;
-  return current_device(dev, sms);
+  L.stream = static_cast<cudaStream_t>(stream);
+  return current_device(L.dev, L.sms);
+}
+
+mlp_status_t check_split(int32_t split) {
+  if (split < 0 || split > MLP_TP_SPLIT_ALL) return fail(MLP_ERR_INVALID_ARG, "split flags %d out of range", split);
+  return MLP_OK;
 }
 
 }  // namespace
@@ -353,110 +399,107 @@ size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t) {
 }
 
 mlp_status_t mlp_tp_fc1_forward(const void* X, const void* A, const void* a, int64_t T, int64_t h, int64_t f,
-                                int32_t t, void* Z, void* H, void* ws, size_t ws_bytes, void* stream) {
+                                int32_t t, void* Z, void* H, void* H_lo, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st = prologue(s, {{X, "X", false}, {A, "A", false}, {a, "a", false}, {Z, "Z", false}, {H, "H", false}},
-                             ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {Z, "Z", false, s.T == 0},
+                                 {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc1_forward(s, X, A, a, Z, H, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc1_forward(s, X, A, a, Z, H, H_lo, ws, L);
 }
 
-mlp_status_t mlp_tp_fc2_forward(const void* H, const void* B, const void* b, int64_t T, int64_t h, int64_t f,
-                                int32_t t, void* Y, void* ws, size_t ws_bytes, void* stream) {
+mlp_status_t mlp_tp_fc2_forward(const void* H, const void* H_lo, const void* B, const void* b, int64_t T, int64_t h,
+                                int64_t f, int32_t t, void* Y, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st = prologue(s, {{H, "H", false}, {B, "B", false}, {b, "b", true}, {Y, "Y", false}}, ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{H, "H", false, s.T == 0}, {H_lo, "H_lo", true, s.T == 0}, {B, "B", false}, {b, "b", true},
+                                 {Y, "Y", false, s.T == 0}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc2_forward(s, H, B, b, Y, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc2_forward(s, H, H_lo, B, b, Y, ws, L);
 }
 
 mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a, const void* B, const void* b, int64_t T,
-                            int64_t h, int64_t f, int32_t t, void* Y, void* Z, void* H, void* ws, size_t ws_bytes,
-                            void* stream) {
+                            int64_t h, int64_t f, int32_t t, int32_t split, void* Y, void* Z, void* H, void* H_lo,
+                            void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st = prologue(s,
-                             {{X, "X", false},
-                              {A, "A", false},
-                              {a, "a", false},
-                              {B, "B", false},
-                              {b, "b", false},
-                              {Y, "Y", false},
-                              {Z, "Z", false},
-                              {H, "H", false}},
-                             ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = check_split(split);
   if (st != MLP_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  st = fc1_forward(s, X, A, a, Z, H, ws, sms, cs);
+  st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
+                    {Y, "Y", false, s.T == 0}, {Z, "Z", false, s.T == 0}, {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}},
+                ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc2_forward(s, H, B, b, Y, ws, sms, cs);
+  st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L);
+  if (st != MLP_OK) return st;
+  return fc2_forward(s, H, (split & MLP_TP_SPLIT_FC2_FORWARD) ? H_lo : nullptr, B, b, Y, ws, L);
 }
 
 mlp_status_t mlp_tp_fc2_backward_data(const void* dY, const void* B, const void* Z, int64_t T, int64_t h, int64_t f,
-                                      int32_t t, void* dH, void* ws, size_t ws_bytes, void* stream) {
+                                      int32_t t, void* dH, void* dH_lo, void* da, void* ws, size_t ws_bytes,
+                                      void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st =
-      prologue(s, {{dY, "dY", false}, {B, "B", false}, {Z, "Z", false}, {dH, "dH", false}}, ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{dY, "dY", false, s.T == 0}, {B, "B", false}, {Z, "Z", false, s.T == 0}, {dH, "dH", false, s.T == 0},
+                                 {dH_lo, "dH_lo", false, s.T == 0}, {da, "da", true}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc2_backward_data(s, dY, B, Z, dH, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L);
 }
 
-mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* dY, int64_t T, int64_t h, int64_t f, int32_t t,
-                                        void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
+mlp_status_t mlp_tp_fc2_backward_weight(const void* H, const void* H_lo, const void* dY, int64_t T, int64_t h,
+                                        int64_t f, int32_t t, void* dB, void* db, void* ws, size_t ws_bytes,
+                                        void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st =
-      prologue(s, {{H, "H", false}, {dY, "dY", false}, {dB, "dB", false}, {db, "db", true}}, ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}, {dY, "dY", false, s.T == 0}, {dB, "dB", false},
+                                 {db, "db", true}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc2_backward_weight(s, H, dY, dB, db, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L);
 }
 
-mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* A, int64_t T, int64_t h, int64_t f, int32_t t,
-                                      void* dX, void* ws, size_t ws_bytes, void* stream) {
+mlp_status_t mlp_tp_fc1_backward_data(const void* dH, const void* dH_lo, const void* A, int64_t T, int64_t h,
+                                      int64_t f, int32_t t, void* dX, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st = prologue(s, {{dH, "dH", false}, {A, "A", false}, {dX, "dX", false}}, ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{dH, "dH", false, s.T == 0}, {dH_lo, "dH_lo", true, s.T == 0}, {A, "A", false}, {dX, "dX", false, s.T == 0}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc1_backward_data(s, dH, A, dX, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc1_backward_data(s, dH, dH_lo, A, dX, ws, L);
 }
 
-mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, int64_t T, int64_t h, int64_t f, int32_t t,
-                                        void* dA, void* da, void* ws, size_t ws_bytes, void* stream) {
+mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const void* dH_lo, int64_t T, int64_t h,
+                                        int64_t f, int32_t t, void* dA, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st =
-      prologue(s, {{X, "X", false}, {dH, "dH", false}, {dA, "dA", false}, {da, "da", true}}, ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = prologue(s, {{X, "X", false, s.T == 0}, {dH, "dH", false, s.T == 0}, {dH_lo, "dH_lo", false, s.T == 0}, {dA, "dA", false}},
+                             ws, ws_bytes, stream, L);
   if (st != MLP_OK) return st;
-  return fc1_backward_weight(s, X, dH, dA, da, ws, sms, static_cast<cudaStream_t>(stream));
+  return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
 }
 
 mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const void* B, const void* Z, const void* H,
-                             int64_t T, int64_t h, int64_t f, int32_t t, void* dX, void* dA, void* da, void* dB,
-                             void* db, void* ws, size_t ws_bytes, void* stream) {
+                             const void* H_lo, int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* dX,
+                             void* dA, void* da, void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
-  int sms = 0;
-  mlp_status_t st = prologue(s,
-                             {{dY, "dY", false},
-                              {X, "X", false},
-                              {A, "A", false},
-                              {B, "B", false},
-                              {Z, "Z", false},
-                              {H, "H", false},
-                              {dX, "dX", false},
-                              {dA, "dA", false},
-                              {da, "da", true},
-                              {dB, "dB", false},
-                              {db, "db", true}},
-                             ws, ws_bytes, sms);
+  Launch L;
+  mlp_status_t st = check_split(split);
   if (st != MLP_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {B, "B", false}, {Z, "Z", false, s.T == 0},
+                    {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
+                    {dB, "dB", false}, {db, "db", true}},
+                ws, ws_bytes, stream, L);
+  if (st != MLP_OK) return st;
   void* dH = static_cast<char*>(ws) + dh_offset();
-  if ((st = fc2_backward_data(s, dY, B, Z, dH, ws, sms, cs)) != MLP_OK) return st;
-  if ((st = fc2_backward_weight(s, H, dY, dB, db, ws, sms, cs)) != MLP_OK) return st;
-  if ((st = fc1_backward_data(s, dH, A, dX, ws, sms, cs)) != MLP_OK) return st;
-  return fc1_backward_weight(s, X, dH, dA, da, ws, sms, cs);
+  void* dH_lo = static_cast<char*>(ws) + dh_lo_offset(s);
+  if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
+  if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
+  if ((st = fc1_backward_data(s, dH, (split & MLP_TP_SPLIT_FC1_BACKWARD_DATA) ? dH_lo : nullptr, A, dX, ws, L)) !=
+      MLP_OK)
+    return st;
+  return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
 }
 
 mlp_status_t mlp_tp_check(void* ws, void* stream) {

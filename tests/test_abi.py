@@ -41,8 +41,8 @@ def test_status_strings(lib):
 
 def test_workspace_bytes(lib):
     n = binding.workspace_bytes(64, 256, 1024, 2)
-    # header 256 + dH 64*1024*2 + one 256-row chunk of max(f,h) fp32 partials
-    assert n == 256 + 64 * 1024 * 2 + 1024 * 4
+    # header 256 + dH pair 2*64*1024*2 + da partials (one 128-row block x 4 quadrants x f fp32)
+    assert n == 256 + 2 * 64 * 1024 * 2 + 4 * 1024 * 4
     assert binding.workspace_bytes(64, 256, 1000, 2) == 0   # f/t not a multiple of 64
     assert binding.workspace_bytes(64, 100, 1024, 2) == 0   # h not a multiple of 64
     assert binding.workspace_bytes(64, 256, 1024, 0) == 0   # t < 1
@@ -53,16 +53,17 @@ FAKE = 1 << 20  # a 16-byte aligned fake address: validation must fail before an
 
 
 def call_fc1(lib, **kw):
-    args = dict(X=FAKE, A=FAKE, a=FAKE, T=64, h=256, f=1024, t=2, Z=FAKE, H=FAKE, ws=FAKE * 2,
+    args = dict(X=FAKE, A=FAKE, a=FAKE, T=64, h=256, f=1024, t=2, Z=FAKE, H=FAKE, H_lo=FAKE, ws=FAKE * 2,
                 ws_bytes=1 << 30, stream=None)
     args.update(kw)
     return lib.mlp_tp_fc1_forward(args["X"], args["A"], args["a"], args["T"], args["h"], args["f"], args["t"],
-                                  args["Z"], args["H"], args["ws"], args["ws_bytes"], args["stream"])
+                                  args["Z"], args["H"], args["H_lo"], args["ws"], args["ws_bytes"], args["stream"])
 
 
 @pytest.mark.parametrize("kw,status,needle", [
     (dict(X=None), 1, "X is NULL"),
     (dict(H=None), 1, "H is NULL"),
+    (dict(H_lo=None), 1, "H_lo is NULL"),
     (dict(t=0), 1, "t=0"),
     (dict(T=-5), 1, "negative"),
     (dict(h=96), 2, "h=96"),
@@ -98,4 +99,10 @@ def test_binding_refuses_cpu_tensors(lib):
     import torch
     x = torch.zeros(64, 256, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
-        binding.mlp_tp_fc1_forward(x, x, x, 64, 256, 1024, 2, x, x, (FAKE, 1 << 30), stream=0)
+        binding.mlp_tp_fc1_forward(x, x, x, 64, 256, 1024, 2, x, x, x, (FAKE, 1 << 30), stream=0)
+
+
+def test_split_flags_are_validated(lib):
+    st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, 1024, 2, 7, FAKE, FAKE, FAKE, FAKE,
+                            FAKE * 2, 1 << 30, None)
+    assert st == 1 and "split" in binding.mlp_tp_last_error()
