@@ -168,6 +168,30 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
                                         void* dA,
                                         void* ws, size_t ws_bytes, void* stream);
 
+/* ----------------------------------------------------- allocation-free */
+
+/* db = sum over rows of dY (the row-parallel layer's bias gradient, as
+ * mlp_tp_fc2_backward_weight computes it) without a workspace.
+ *
+ * The pages describe nothing like this; it exists for callers that cannot
+ * allocate device memory: code that must run from a fixed, pre-planned
+ * memory budget (a serving process whose pool already owns every byte of
+ * HBM), or a host framework whose plugin interface hands over only the
+ * input and output pointers, with no scratch and no allocator.  The fp32
+ * partial sums go to a static device array of 2^20 floats (4 MiB) inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Shapes with ceil(T/256)·h > 2^20 are rejected with
+ * MLP_ERR_UNSUPPORTED_SHAPE (use mlp_tp_fc2_backward_weight then).
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array: calls whose
+ * work overlaps on the GPU (different streams, or several host threads
+ * without ordering) race on it; calls ordered on one stream do not.  No
+ * call allocates or frees memory.  Same pointer, alignment and device rules
+ * as the other entry points; dY may be NULL when T == 0 (db is zero-filled). */
+mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, int64_t h, void* db, void* stream);
+
 /* ------------------------------------------------------------ diagnostics */
 
 /* Synchronises `stream`, then reads and clears the device status word in

@@ -42,6 +42,7 @@ _SIGS = {
     "mlp_tp_fc2_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_fc1_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_fc1_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_bias_grad_noalloc": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "mlp_tp_check": ([_P, _P], ctypes.c_int),
     "mlp_tp_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "mlp_tp_last_error": ([], ctypes.c_char_p),
@@ -193,6 +194,11 @@ def mlp_tp_fc1_backward_weight(X, dH, dH_lo, T, h, f, t, dA, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_fc1_backward_weight(_addr(X, "X"), _addr(dH, "dH"), _addr(dH_lo, "dH_lo"), T, h, f, t,
                                             _addr(dA, "dA"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db, stream=None):
+    """db = Σ_rows dY with no workspace (the library's static scratch)."""
+    _check(lib().mlp_tp_fc2_bias_grad_noalloc(_addr(dY, "dY", T == 0), T, h, _addr(db, "db"), _stream(stream)))
 
 
 def mlp_tp_check(ws, stream=None):

@@ -542,3 +542,54 @@ void mlp_tp_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull 
 void mlp_tp_set_debug_flags(uint32_t flags) { g_debug_flags.store(flags); }
 
 }  // extern "C"
+
+// ============================================================ allocation-free
+// db = Σ_rows dY for callers that cannot allocate device memory and so have
+// no workspace to hand over (see mlp_tp_fc2_bias_grad_noalloc in the
+// header).  The fp32 partial sums live in this file-scope device array, which
+// every GPU that loads the library holds until the process exits.
+namespace {
+
+constexpr size_t NOALLOC_MAX_PARTIALS = size_t(1) << 20;  // 4 MiB of fp32
+static __device__ __align__(256) float g_noalloc_partials[NOALLOC_MAX_PARTIALS];
+
+// Host code may not use g_noalloc_partials directly (on the host it only
+// names a stand-in); its device address is looked up once per device, with
+// that device current.
+float* g_noalloc_ptr[64] = {};
+std::mutex g_noalloc_mu;
+
+mlp_status_t noalloc_scratch(int dev, float** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static column-sum scratch)");
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLP_OK;
+}
+
+}  // namespace
+
+extern "C" mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, int64_t h, void* db, void* stream) {
+  if (T < 0 || h < 0) return fail(MLP_ERR_INVALID_ARG, "negative size T=%lld h=%lld", (long long)T, (long long)h);
+  if (h < 64 || h % 64 != 0 || T > (int64_t(1) << 31) - 1 || h > (int64_t(1) << 31) - 1)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "h=%lld must be a positive multiple of 64 and T, h < 2^31", (long long)h);
+  const size_t need = colsum_chunks(T) * static_cast<size_t>(h);
+  if (need > NOALLOC_MAX_PARTIALS)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE,
+                "T=%lld, h=%lld needs %zu fp32 partial sums; the allocation-free path holds at most %zu "
+                "(ceil(T/%d)*h <= %zu); use mlp_tp_fc2_backward_weight with a workspace instead",
+                (long long)T, (long long)h, need, NOALLOC_MAX_PARTIALS, COLSUM_ROWS_PER_CHUNK, NOALLOC_MAX_PARTIALS);
+  mlp_status_t st = check_ptrs({{dY, "dY", false, T == 0}, {db, "db", false}});
+  if (st != MLP_OK) return st;
+  int dev = 0, sms = 0;
+  if ((st = current_device(dev, sms)) != MLP_OK) return st;
+  float* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != MLP_OK) return st;
+  // Pass 1 overwrites every partial it reads back in pass 2, so nothing left
+  // in the array by an earlier call is ever used.
+  return launch_colsum(dY, T, h, db, scratch, static_cast<cudaStream_t>(stream));
+}
