@@ -3,15 +3,23 @@
 //
 //   D[M,N] = sum_k Aop[M,k] · Bop[k,N]   (bf16 in, fp32 accumulate in TMEM)
 //
-// One CTA per SM walks a static list of 128x256 output tiles.  Warp roles:
+// Persistent grid, one CTA per SM.  In the default pair mode two CTAs of a
+// cluster share each 256x256 output tile through the 2-SM tensor-core
+// instruction (cta_group::2): CTA r of the pair owns rows [128r, 128r+128)
+// of the tile (its half of the A operand and of the TMEM accumulator) and
+// columns [128r, 128r+128) of the B operand, so each SM streams half of B
+// instead of all of it.  In single mode a CTA owns a 128x256 tile alone.
+// Warp roles (per CTA):
 //   warp 0      TMA producer: fills a ring of STAGES shared-memory stages
-//               (A tile 128x64, B tile 256x64, 128-byte swizzle) and arms a
-//               "full" mbarrier with the expected byte count;
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators),
-//               and one thread issues tcgen05.mma (M=128, N=256, K=16) per
-//               16-wide K slice, committing each stage back to its "empty"
-//               barrier and each finished accumulator to a "tmem full"
-//               barrier;
+//               (its A rows x 64 and its B rows x 64, 128-byte swizzle); the
+//               pair leader arms the "full" mbarrier with the byte count of
+//               both CTAs' loads, which all complete on the leader's barrier;
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators
+//               per CTA); on the leader, one thread issues tcgen05.mma
+//               (M=256 across the pair, or 128 alone; N=256; K=16) per
+//               16-wide K slice, committing each stage back to the "empty"
+//               barriers of both CTAs and each finished accumulator to their
+//               "tmem full" barriers;
 //   warps 2-9   epilogue: tcgen05.ld the accumulator (one row per thread,
 //               32 columns per load), apply the fused math, store to global
 //               memory, release the accumulator.
@@ -52,19 +60,35 @@
 
 namespace mlptp {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;  // accumulator rows per CTA
+constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int MN_BOX_BYTES = 64 * BK * 2;   // one 64x64 bf16 box, 8 KB
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int CTL_BYTES = 1024;
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + CTL_BYTES + 1024;  // + alignment slack
+
+// Shared-memory pipeline depth (stages of BK-wide K slices in flight).
+#ifndef MLPTP_PAIR_STAGES
+#define MLPTP_PAIR_STAGES 6
+#endif
+#ifndef MLPTP_SINGLE_STAGES
+#define MLPTP_SINGLE_STAGES 4
+#endif
+
+template <bool PAIR>
+struct TileCfg {
+  static constexpr int CTAS = PAIR ? 2 : 1;
+  static constexpr int TILE_M = BM * CTAS;                    // output rows per tile
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;            // B operand rows held by one CTA
+  static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // one CTA's share of a stage
+  static constexpr int STAGES = PAIR ? MLPTP_PAIR_STAGES : MLPTP_SINGLE_STAGES;
+  static_assert(STAGES <= 8, "control block holds at most 8 stages");
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CTL_BYTES + 1024;  // + alignment slack
+};
 
 constexpr unsigned int STATUS_TIMEOUT = 7u;
 
@@ -94,9 +118,10 @@ struct GemmMaps {
   CUtensorMap b[2];
 };
 
+constexpr int MAX_STAGES = 8;
 struct GemmCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t mma_done;
@@ -242,29 +267,35 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- kernel
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+  using Cfg = TileCfg<PAIR>;
+  constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(smem + STAGES * STAGE_BYTES);
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(smem + STAGES * Cfg::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_cta_rank() : 0u;  // position in the CTA pair
+  const bool leader = rank == 0;
+  const int cluster_id = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int num_clusters = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctl->full[s], 1);
-      mbar_init(&ctl->empty[s], 1);
+      mbar_init(&ctl->full[s], 1);   // one arrival: the leader's expect_tx
+      mbar_init(&ctl->empty[s], 1);  // one arrival: the leader's MMA commit
     }
 #pragma unroll
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctl->tfull[a], 1);
-      mbar_init(&ctl->tempty[a], NUM_EPI_WARPS);
+      mbar_init(&ctl->tempty[a], NUM_EPI_WARPS * Cfg::CTAS);  // every epilogue warp of the pair
     }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort = 0;
@@ -278,11 +309,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
@@ -294,13 +334,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_phase = 0;  // per stage: filled at least once / parity of last fill
+      uint32_t issued_mask = 0, issued_phase = 0;  // per stage: armed at least once / parity of last arming
       bool ok = true;
       bool first = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
         int mb, nb;
         tile_coords(tile, p, mb, nb);
-        const int m0 = mb * BM, n0 = nb * BN;
+        const int m0 = mb * Cfg::TILE_M + static_cast<int>(rank) * BM;   // this CTA's A rows
+        const int n0 = nb * BN + static_cast<int>(rank) * Cfg::B_ROWS;   // this CTA's B rows
         for (int s = 0; ok && s < p.shards; ++s) {
           for (int i = 0; i < kb_per_unit; ++i) {
             if ((p.debug_flags & 1u) && !first) {
@@ -317,24 +358,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int k0 = (s * p.kblocks_per_shard + (i - part * p.kblocks_per_shard)) * BK;
             const CUtensorMap* ma = &maps.a[part];
             const CUtensorMap* mbp = &maps.b[part];
-            const uint32_t fb = smem_u32(&ctl->full[stage]);
-            mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
             const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
-            const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
-            if (A_MN) {
-              tma_load_2d(a_dst, ma, fb, m0, k0);
-              tma_load_2d(a_dst + MN_BOX_BYTES, ma, fb, m0 + 64, k0);
-            } else {
-              tma_load_2d(a_dst, ma, fb, k0, m0);
-            }
-            if (B_MN) {
+            const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+            if constexpr (PAIR) {
+              const uint32_t fb = map_shared_to_cta(smem_u32(&ctl->full[stage]), 0u);
+              if (leader) {
+                mbar_arrive_expect_tx(&ctl->full[stage], Cfg::CTAS * Cfg::STAGE_BYTES);
+                issued_mask |= 1u << stage;
+                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+              }
+              if (A_MN) {
+                tma_load_2d_pair(a_dst, ma, fb, m0, k0);
+                tma_load_2d_pair(a_dst + MN_BOX_BYTES, ma, fb, m0 + 64, k0);
+              } else {
+                tma_load_2d_pair(a_dst, ma, fb, k0, m0);
+              }
+              if (B_MN) {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
+                for (int j = 0; j < Cfg::B_ROWS / 64; ++j)
+                  tma_load_2d_pair(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
+              } else {
+                tma_load_2d_pair(b_dst, mbp, fb, k0, n0);
+              }
             } else {
-              tma_load_2d(b_dst, mbp, fb, k0, n0);
+              const uint32_t fb = smem_u32(&ctl->full[stage]);
+              mbar_arrive_expect_tx(&ctl->full[stage], Cfg::STAGE_BYTES);
+              issued_mask |= 1u << stage;
+              issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+              if (A_MN) {
+                tma_load_2d(a_dst, ma, fb, m0, k0);
+                tma_load_2d(a_dst + MN_BOX_BYTES, ma, fb, m0 + 64, k0);
+              } else {
+                tma_load_2d(a_dst, ma, fb, k0, m0);
+              }
+              if (B_MN) {
+#pragma unroll
+                for (int j = 0; j < Cfg::B_ROWS / 64; ++j)
+                  tma_load_2d(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
+              } else {
+                tma_load_2d(b_dst, mbp, fb, k0, n0);
+              }
             }
-            issued_mask |= 1u << stage;
-            issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -342,20 +406,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // No TMA write may still be landing in this CTA's shared memory when it
-      // exits: wait for the last fill of every stage (immediate when the
-      // tensor-core warp already consumed it).
+      // No TMA write may still be landing in shared memory when the CTAs
+      // exit: the barrier owner waits for the last arming of every stage
+      // (immediate when the tensor-core warp already consumed it).  In pair
+      // mode the leader's barriers also count the peer's copies.
       for (int s = 0; s < STAGES; ++s)
         if (issued_mask & (1u << s)) mbar_drain(&ctl->full[s], (issued_phase >> s) & 1u, budget);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(Cfg::TILE_M, BN, A_MN, B_MN);
+      constexpr uint16_t PAIR_MASK = 0x3;
       int stage = 0;
       uint32_t phase = 0, unit = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
         for (int s = 0; ok && s < p.shards; ++s, ++unit) {
           const uint32_t acc = unit & 1u, acc_phase = (unit >> 1) & 1u;
           if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, abort_flag, budget)) {
@@ -373,7 +439,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_fence_after_sync();
             const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
-            const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+            const uint32_t b_base = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
               // K-major: the 16-wide K slice is 32 bytes further along each
@@ -384,20 +450,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
               const uint64_t bd = B_MN ? smem_desc_sw128(b_base + k * 2048, MN_BOX_BYTES, 1024)
                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
-              mma_bf16_ss(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+              if constexpr (PAIR) {
+                mma_bf16_pair(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+              } else {
+                mma_bf16_ss(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+              }
             }
-            mma_commit(&ctl->empty[stage]);
+            if constexpr (PAIR) {
+              mma_commit_pair_multicast(&ctl->empty[stage], PAIR_MASK);
+            } else {
+              mma_commit(&ctl->empty[stage]);
+            }
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
             }
           }
           if (!ok) break;
-          mma_commit(&ctl->tfull[acc]);
+          if constexpr (PAIR) {
+            mma_commit_pair_multicast(&ctl->tfull[acc], PAIR_MASK);
+          } else {
+            mma_commit(&ctl->tfull[acc]);
+          }
         }
       }
       // Every MMA this thread issued must finish before TMEM is released.
-      mma_commit(&ctl->mma_done);
+      if constexpr (PAIR) {
+        mma_commit_pair(&ctl->mma_done);
+      } else {
+        mma_commit(&ctl->mma_done);
+      }
       mbar_drain(&ctl->mma_done, 0u, budget);
     }
   } else {
@@ -405,12 +487,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int ew = warp - 2;
     const int q = warp & 3;     // TMEM lane quadrant this warp may access
     const int half = ew >> 2;   // 128-column half of the tile
+    // the MMA issuer's "accumulator drained" barriers (in the leader CTA)
+    uint32_t tempty_addr[2] = {0u, 0u};
+    if constexpr (PAIR) {
+      tempty_addr[0] = map_shared_to_cta(smem_u32(&ctl->tempty[0]), 0u);
+      tempty_addr[1] = map_shared_to_cta(smem_u32(&ctl->tempty[1]), 0u);
+    }
     uint32_t unit = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
       int mb, nb;
       tile_coords(tile, p, mb, nb);
-      const int row = mb * BM + q * 32 + lane;
+      const int row_block = mb * Cfg::CTAS + static_cast<int>(rank);  // this CTA's 128-row block
+      const int row = row_block * BM + q * 32 + lane;
       const bool row_ok = row < p.M;
       const size_t row_off = static_cast<size_t>(row) * static_cast<size_t>(p.N);
       float sum[EPI == EPI_SHARD_SUM ? 128 : 1];
@@ -465,7 +554,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (p.colsum != nullptr) {
               const float cs = warp_column_sums(dh);
-              p.colsum[static_cast<size_t>(mb * 4 + q) * p.N + col + lane] = cs;
+              p.colsum[static_cast<size_t>(row_block * 4 + q) * p.N + col + lane] = cs;
             }
           } else if constexpr (EPI == EPI_STORE) {
             uint32_t op[16];
@@ -498,16 +587,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+        if (lane == 0) {
+          if constexpr (PAIR) {
+            mbar_arrive_cluster(tempty_addr[acc]);
+          } else {
+            mbar_arrive(&ctl->tempty[acc]);
+          }
+        }
       }
     }
   }
 
-  __syncthreads();
+  // Both CTAs of a pair stay resident until all remote arrivals and
+  // multicast commits addressed to them have landed.
+  tc_fence_before_sync();
+  if constexpr (PAIR) {
+    cluster_sync_all();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    } else {
+      tmem_dealloc(tmem_base, TMEM_COLS);
+    }
   }
 }
 

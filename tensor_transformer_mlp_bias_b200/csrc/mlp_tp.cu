@@ -66,7 +66,16 @@ mlp_status_t check_shape(const Shape& s) {
 }
 
 size_t colsum_chunks(int64_t R) { return static_cast<size_t>((R + COLSUM_ROWS_PER_CHUNK - 1) / COLSUM_ROWS_PER_CHUNK); }
-size_t gemm_row_blocks(int64_t R) { return static_cast<size_t>((R + BM - 1) / BM); }
+// The GEMMs run on CTA pairs (2-SM tensor-core instructions, 256-row tiles).
+#ifndef MLPTP_USE_PAIR
+#define MLPTP_USE_PAIR 1
+#endif
+constexpr bool kPair = MLPTP_USE_PAIR != 0;
+using TileShape = TileCfg<kPair>;
+// 128-row blocks that a GEMM over R rows covers (whole tiles).
+size_t gemm_row_blocks(int64_t R) {
+  return static_cast<size_t>((R + TileShape::TILE_M - 1) / TileShape::TILE_M) * TileShape::CTAS;
+}
 
 // Workspace layout: [status header | dH | dH_lo | fp32 column-sum partials].
 size_t pair_bytes(const Shape& s) { return align_up(static_cast<size_t>(s.T * s.f * 2), 256); }
@@ -206,16 +215,38 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
 
 // One opt-in per kernel instantiation and device (the static state is per
 // template instance).
-template <bool A_MN, bool B_MN, int EPI>
-mlp_status_t ensure_smem_attr(int dev) {
+template <bool A_MN, bool B_MN, int EPI, bool PAIR>
+mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
   static std::mutex mu;
   static uint64_t done_mask = 0;
-  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI>;
+  static int clusters[64] = {};
+  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR>;
   std::lock_guard<std::mutex> lk(mu);
-  if (done_mask & (1ull << dev)) return MLP_OK;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
-  done_mask |= 1ull << dev;
+  if (!(done_mask & (1ull << dev))) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<PAIR>::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+    int n = sms / TileCfg<PAIR>::CTAS;
+    if (PAIR) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * n));
+      cfg.blockDim = dim3(NUM_THREADS);
+      cfg.dynamicSmemBytes = TileCfg<PAIR>::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int q = 0;
+      if (cudaOccupancyMaxActiveClusters(&q, kernel, &cfg) == cudaSuccess && q > 0 && q < n) n = q;
+      cudaGetLastError();  // a failed occupancy query leaves no sticky error; keep the SM-count bound
+    }
+    clusters[dev] = n;
+    done_mask |= 1ull << dev;
+  }
+  *max_clusters = clusters[dev];
   return MLP_OK;
 }
 
@@ -225,14 +256,15 @@ struct Launch {
   cudaStream_t stream;
 };
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR = kPair>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
+  using Cfg = TileCfg<PAIR>;
   if (g.M == 0 || g.N == 0) return MLP_OK;
   GemmMaps maps;
   for (int i = 0; i < 2; ++i) {
     mlp_status_t st = make_operand_map(&maps.a[i], g.a.p[i], A_MN, g.M, g.K, BM, name);
     if (st != MLP_OK) return st;
-    st = make_operand_map(&maps.b[i], g.b.p[i], B_MN, g.N, g.K, BN, name);
+    st = make_operand_map(&maps.b[i], g.b.p[i], B_MN, g.N, g.K, Cfg::B_ROWS, name);
     if (st != MLP_OK) return st;
   }
   p.M = static_cast<int>(g.M);
@@ -240,18 +272,31 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.shards = g.shards;
   p.parts = g.parts;
   p.kblocks_per_shard = static_cast<int>((g.K / g.shards + BK - 1) / BK);
-  p.m_blocks = static_cast<int>((g.M + BM - 1) / BM);
+  p.m_blocks = static_cast<int>((g.M + Cfg::TILE_M - 1) / Cfg::TILE_M);
   p.n_blocks = static_cast<int>((g.N + BN - 1) / BN);
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
   p.budget_ns = g_budget_ns.load();
   p.debug_flags = g_debug_flags.load();
 
-  mlp_status_t st = ensure_smem_attr<A_MN, B_MN, EPI>(L.dev);
+  int max_clusters = 0;
+  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR>(L.dev, L.sms, &max_clusters);
   if (st != MLP_OK) return st;
-  const int grid = p.num_tiles < L.sms ? p.num_tiles : L.sms;
-  mlp_gemm_kernel<A_MN, B_MN, EPI><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, L.stream>>>(maps, p);
-  cudaError_t e = cudaGetLastError();
+  const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = Cfg::CTAS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CTAS));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = L.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR>, maps, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
   return MLP_OK;
