@@ -358,10 +358,15 @@ def main():
     products["fc1_backward_data"] += 1 if split & 2 else 0
     gemm_flops = 2.0 * T * h * f * products[dom]
     achieved = gemm_flops / (stage_ms[dom] * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    # The step is short (a few ms, a few hundred ms in all) and the clocks stay
+    # near their maximum, so the burst figure (cuBLAS timed alone at the same
+    # clocks) is the like-for-like peak; the sustained figure is reported too.
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     roofline = {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved,
                 "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "peak_source": f"{peak_src} bf16_tflops (burst; clocks in this run: see clocks)",
+                "frac_of_sustained": achieved / peak_sustained,
                 "traffic": traffic_for(dom, wl, t),
                 "algorithmic_flops_per_launch": gemm_flops, "avg_launch_ms": stage_ms[dom]}
 

@@ -78,14 +78,29 @@ constexpr int CTL_BYTES = 1024;
 #define MLPTP_SINGLE_STAGES 4
 #endif
 
-template <bool PAIR>
+#ifndef MLPTP_WIDE_STAGES
+#define MLPTP_WIDE_STAGES 4
+#endif
+
+// Tile shape.  TN is the number of output columns per tile: 256 (one MMA
+// width, two TMEM accumulators so the epilogue overlaps the next tile) or
+// 512 (pair mode only: two MMA widths side by side, one accumulator filling
+// all 512 TMEM columns).  The wide tile reads 25% fewer operand bytes per
+// FLOP from L2, which is what bounds these GEMMs without TMA multicast.
+template <bool PAIR, int TN = 256>
 struct TileCfg {
+  static_assert(TN == 256 || (TN == 512 && PAIR), "wide tiles need a CTA pair");
   static constexpr int CTAS = PAIR ? 2 : 1;
   static constexpr int TILE_M = BM * CTAS;                    // output rows per tile
-  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;            // B operand rows held by one CTA
+  static constexpr int TILE_N = TN;
+  static constexpr int WIDTHS = TN / BN;                       // MMA widths per tile
+  static constexpr int ACCS = TN == 256 ? 2 : 1;               // TMEM accumulators (double-buffered or not)
+  static constexpr int SUB_ROWS = PAIR ? BN / 2 : BN;          // B rows per CTA per MMA width
+  static constexpr int B_ROWS = SUB_ROWS * WIDTHS;             // B operand rows held by one CTA
+  static constexpr int SUB_BYTES = SUB_ROWS * BK * 2;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // one CTA's share of a stage
-  static constexpr int STAGES = PAIR ? MLPTP_PAIR_STAGES : MLPTP_SINGLE_STAGES;
+  static constexpr int STAGES = TN == 512 ? MLPTP_WIDE_STAGES : (PAIR ? MLPTP_PAIR_STAGES : MLPTP_SINGLE_STAGES);
   static_assert(STAGES <= 8, "control block holds at most 8 stages");
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CTL_BYTES + 1024;  // + alignment slack
 };
@@ -267,10 +282,12 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- kernel
-template <bool A_MN, bool B_MN, int EPI, bool PAIR>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
-  using Cfg = TileCfg<PAIR>;
+  using Cfg = TileCfg<PAIR, TN>;
+  static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
+  constexpr int ACCS = Cfg::ACCS;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -293,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ctl->empty[s], 1);  // one arrival: the leader's MMA commit
     }
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < ACCS; ++a) {
       mbar_init(&ctl->tfull[a], 1);
       mbar_init(&ctl->tempty[a], NUM_EPI_WARPS * Cfg::CTAS);  // every epilogue warp of the pair
     }
@@ -340,8 +357,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
         int mb, nb;
         tile_coords(tile, p, mb, nb);
-        const int m0 = mb * Cfg::TILE_M + static_cast<int>(rank) * BM;   // this CTA's A rows
-        const int n0 = nb * BN + static_cast<int>(rank) * Cfg::B_ROWS;   // this CTA's B rows
+        const int m0 = mb * Cfg::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
+        // this CTA's B rows for MMA width w start at n0 + w * BN
+        const int n0 = nb * Cfg::TILE_N + static_cast<int>(rank) * Cfg::SUB_ROWS;
         for (int s = 0; ok && s < p.shards; ++s) {
           for (int i = 0; i < kb_per_unit; ++i) {
             if ((p.debug_flags & 1u) && !first) {
@@ -373,12 +391,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               } else {
                 tma_load_2d_pair(a_dst, ma, fb, k0, m0);
               }
-              if (B_MN) {
 #pragma unroll
-                for (int j = 0; j < Cfg::B_ROWS / 64; ++j)
-                  tma_load_2d_pair(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
-              } else {
-                tma_load_2d_pair(b_dst, mbp, fb, k0, n0);
+              for (int w = 0; w < Cfg::WIDTHS; ++w) {
+                if (B_MN) {
+#pragma unroll
+                  for (int j = 0; j < Cfg::SUB_ROWS / 64; ++j)
+                    tma_load_2d_pair(b_dst + w * Cfg::SUB_BYTES + j * MN_BOX_BYTES, mbp, fb, n0 + w * BN + 64 * j, k0);
+                } else {
+                  tma_load_2d_pair(b_dst + w * Cfg::SUB_BYTES, mbp, fb, k0, n0 + w * BN);
+                }
               }
             } else {
               const uint32_t fb = smem_u32(&ctl->full[stage]);
@@ -391,12 +412,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               } else {
                 tma_load_2d(a_dst, ma, fb, k0, m0);
               }
-              if (B_MN) {
 #pragma unroll
-                for (int j = 0; j < Cfg::B_ROWS / 64; ++j)
-                  tma_load_2d(b_dst + j * MN_BOX_BYTES, mbp, fb, n0 + 64 * j, k0);
-              } else {
-                tma_load_2d(b_dst, mbp, fb, k0, n0);
+              for (int w = 0; w < Cfg::WIDTHS; ++w) {
+                if (B_MN) {
+#pragma unroll
+                  for (int j = 0; j < Cfg::SUB_ROWS / 64; ++j)
+                    tma_load_2d(b_dst + w * Cfg::SUB_BYTES + j * MN_BOX_BYTES, mbp, fb, n0 + w * BN + 64 * j, k0);
+                } else {
+                  tma_load_2d(b_dst + w * Cfg::SUB_BYTES, mbp, fb, k0, n0 + w * BN);
+                }
               }
             }
             if (++stage == STAGES) {
@@ -423,14 +447,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
         for (int s = 0; ok && s < p.shards; ++s, ++unit) {
-          const uint32_t acc = unit & 1u, acc_phase = (unit >> 1) & 1u;
+          const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
           if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, abort_flag, budget)) {
             record_timeout(p, abort_flag, 0x200u);
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t d_tmem = tmem_base + acc * BN;
+          const uint32_t d_tmem = tmem_base + acc * BN;  // ACCS == 1: widths at columns 0 and 256
           for (int i = 0; i < kb_per_unit; ++i) {
             if (!mbar_wait(&ctl->full[stage], phase, abort_flag, budget)) {
               record_timeout(p, abort_flag, 0x300u);
@@ -448,12 +472,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               // further; 64-wide MN blocks are one 8 KB box apart.
               const uint64_t ad = A_MN ? smem_desc_sw128(a_base + k * 2048, MN_BOX_BYTES, 1024)
                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
-              const uint64_t bd = B_MN ? smem_desc_sw128(b_base + k * 2048, MN_BOX_BYTES, 1024)
-                                       : smem_desc_sw128(b_base + k * 32, 16, 1024);
-              if constexpr (PAIR) {
-                mma_bf16_pair(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
-              } else {
-                mma_bf16_ss(d_tmem, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+#pragma unroll
+              for (int w = 0; w < Cfg::WIDTHS; ++w) {
+                const uint32_t bw = b_base + w * Cfg::SUB_BYTES;
+                const uint64_t bd = B_MN ? smem_desc_sw128(bw + k * 2048, MN_BOX_BYTES, 1024)
+                                         : smem_desc_sw128(bw + k * 32, 16, 1024);
+                if constexpr (PAIR) {
+                  mma_bf16_pair(d_tmem + w * BN, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+                } else {
+                  mma_bf16_ss(d_tmem + w * BN, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+                }
               }
             }
             if constexpr (PAIR) {
@@ -486,12 +514,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int q = warp & 3;     // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;   // 128-column half of the tile
+    const int half = ew >> 2;   // column half of the tile (TN/2 columns)
+    constexpr int HALF_COLS = Cfg::TILE_N / 2;
     // the MMA issuer's "accumulator drained" barriers (in the leader CTA)
     uint32_t tempty_addr[2] = {0u, 0u};
     if constexpr (PAIR) {
-      tempty_addr[0] = map_shared_to_cta(smem_u32(&ctl->tempty[0]), 0u);
-      tempty_addr[1] = map_shared_to_cta(smem_u32(&ctl->tempty[1]), 0u);
+#pragma unroll
+      for (int a = 0; a < ACCS; ++a) tempty_addr[a] = map_shared_to_cta(smem_u32(&ctl->tempty[a]), 0u);
     }
     uint32_t unit = 0;
     bool ok = true;
@@ -504,17 +533,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const size_t row_off = static_cast<size_t>(row) * static_cast<size_t>(p.N);
       float sum[EPI == EPI_SHARD_SUM ? 128 : 1];
       for (int s = 0; s < p.shards; ++s, ++unit) {
-        const uint32_t acc = unit & 1u, acc_phase = (unit >> 1) & 1u;
+        const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
         if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort_flag, budget)) {
           record_timeout(p, abort_flag, 0x400u);
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t t_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * 128;
+        const uint32_t t_addr =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * HALF_COLS;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = nb * BN + half * 128 + c * 32;
+        for (int c = 0; c < HALF_COLS / 32; ++c) {
+          const int col = nb * Cfg::TILE_N + half * HALF_COLS + c * 32;
           if (col >= p.N) continue;  // warp-uniform: ragged last column block
           uint32_t r[32];
           tmem_load_32cols(t_addr + c * 32, r);
