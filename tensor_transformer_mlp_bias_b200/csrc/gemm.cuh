@@ -70,24 +70,26 @@ constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int CTL_BYTES = 1024;
 
-// Shared-memory pipeline depth (stages of BK-wide K slices in flight).
-#ifndef MLPTP_PAIR_STAGES
-#define MLPTP_PAIR_STAGES 6
-#endif
-#ifndef MLPTP_SINGLE_STAGES
-#define MLPTP_SINGLE_STAGES 4
-#endif
+enum Epi : int { EPI_BIAS_GELU = 0, EPI_SHARD_SUM = 1, EPI_GELU_GRAD = 2, EPI_STORE = 3 };
 
-#ifndef MLPTP_WIDE_STAGES
-#define MLPTP_WIDE_STAGES 4
-#endif
+// Epilogue staging per epilogue warp: one 32x32 tile per output, laid out
+// for the TMA store (bf16: 64-byte rows, 64-byte swizzle; fp32: 128-byte
+// rows, 128-byte swizzle).
+constexpr int EPI_BF16_TILE = 32 * 32 * 2;
+constexpr int EPI_F32_TILE = 32 * 32 * 4;
+__host__ __device__ constexpr int epi_warp_bytes(int epi) {
+  return epi == EPI_BIAS_GELU ? EPI_F32_TILE + 2 * EPI_BF16_TILE
+                              : (epi == EPI_GELU_GRAD ? 2 * EPI_BF16_TILE : EPI_BF16_TILE);
+}
 
 // Tile shape.  TN is the number of output columns per tile: 256 (one MMA
 // width, two TMEM accumulators so the epilogue overlaps the next tile) or
 // 512 (pair mode only: two MMA widths side by side, one accumulator filling
 // all 512 TMEM columns).  The wide tile reads 25% fewer operand bytes per
 // FLOP from L2, which is what bounds these GEMMs without TMA multicast.
-template <bool PAIR, int TN = 256>
+// STAGES is the shared-memory pipeline depth (BK-wide K slices in flight):
+// as many as fit beside the epilogue staging.
+template <bool PAIR, int TN, int EPI>
 struct TileCfg {
   static_assert(TN == 256 || (TN == 512 && PAIR), "wide tiles need a CTA pair");
   static constexpr int CTAS = PAIR ? 2 : 1;
@@ -100,14 +102,16 @@ struct TileCfg {
   static constexpr int SUB_BYTES = SUB_ROWS * BK * 2;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // one CTA's share of a stage
-  static constexpr int STAGES = TN == 512 ? MLPTP_WIDE_STAGES : (PAIR ? MLPTP_PAIR_STAGES : MLPTP_SINGLE_STAGES);
-  static_assert(STAGES <= 8, "control block holds at most 8 stages");
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CTL_BYTES + 1024;  // + alignment slack
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * epi_warp_bytes(EPI);
+  static constexpr int SMEM_LIMIT = 227 * 1024;
+  static constexpr int FIXED = EPI_BYTES + CTL_BYTES + 1024;   // + alignment slack
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static_assert(STAGES >= 3, "pipeline too shallow");
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
 };
 
 constexpr unsigned int STATUS_TIMEOUT = 7u;
-
-enum Epi : int { EPI_BIAS_GELU = 0, EPI_SHARD_SUM = 1, EPI_GELU_GRAD = 2, EPI_STORE = 3 };
 
 struct GemmParams {
   int M, N;
@@ -118,7 +122,7 @@ struct GemmParams {
   __nv_bfloat16* out0;        // H_hi | Y | dH_hi | dX | dA | dB
   __nv_bfloat16* out1;        // H_lo (EPI_BIAS_GELU) | dH_lo (EPI_GELU_GRAD)
   float* out_f32;             // Z (EPI_BIAS_GELU)
-  float* colsum;              // [m_blocks*4, N] column sums of dH (EPI_GELU_GRAD), may be null
+  float* colsum;              // [row blocks*4, N] column sums of dH (EPI_GELU_GRAD), may be null
   const __nv_bfloat16* bias;  // a (EPI_BIAS_GELU) or b (EPI_SHARD_SUM), may be null for the latter
   const float* aux;           // Z (EPI_GELU_GRAD)
   unsigned int* status;       // device status word pair in the workspace
@@ -127,10 +131,12 @@ struct GemmParams {
 };
 
 // Tensor maps of the operands, one per K part (part 1 repeats part 0 for an
-// operand that is not split).
+// operand that is not split), and of the outputs (32x32 store boxes):
+// out[0] = out0, out[1] = out1 (bf16), out[2] = out_f32.
 struct GemmMaps {
   CUtensorMap a[2];
   CUtensorMap b[2];
+  CUtensorMap out[3];
 };
 
 constexpr int MAX_STAGES = 8;
@@ -247,17 +253,23 @@ __device__ __forceinline__ void load_f32x32(const float* src, float (&dst)[32]) 
   }
 }
 
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
+// Row `r` (this lane) of a 32x32 bf16 staging tile: 64-byte rows, 16-byte
+// chunk j stored at chunk j ^ ((r >> 1) & 3) (the TMA 64-byte swizzle; the
+// tile is 512-byte aligned), so a warp's 16-byte stores hit every bank.
+__device__ __forceinline__ void stage_bf16x32(uint32_t tile, int r, const uint32_t (&packed)[16]) {
 #pragma unroll
-  for (int v = 0; v < 4; ++v)
-    d[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+  for (int j = 0; j < 4; ++j)
+    st_shared_v4(tile + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                 packed[4 * j + 3]);
 }
 
-__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
-  float4* d = reinterpret_cast<float4*>(dst);
+// Row `r` of a 32x32 fp32 staging tile: 128-byte rows, chunk j stored at
+// chunk j ^ (r & 7) (the TMA 128-byte swizzle; the tile is 1024-byte aligned).
+__device__ __forceinline__ void stage_f32x32(uint32_t tile, int r, const float (&v)[32]) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(tile + r * 128 + ((j ^ (r & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                 __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
 }
 
 // Column sums over the warp's 32 rows: lane r holds row r's 32 values; on
@@ -285,7 +297,7 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
-  using Cfg = TileCfg<PAIR, TN>;
+  using Cfg = TileCfg<PAIR, TN, EPI>;
   static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
   constexpr int ACCS = Cfg::ACCS;
   constexpr int STAGES = Cfg::STAGES;
@@ -294,7 +306,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * Cfg::STAGE_BYTES;  // 1024-aligned: STAGE_BYTES is a multiple of 1024
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(sEpi + Cfg::EPI_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -517,6 +530,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = ew >> 2;   // column half of the tile (TN/2 columns)
     constexpr int HALF_COLS = Cfg::TILE_N / 2;
     // the MMA issuer's "accumulator drained" barriers (in the leader CTA)
+    // this warp's staging tiles: [fp32 (EPI_BIAS_GELU)] [bf16 out0] [bf16 out1]
+    const uint32_t stage_base = smem_u32(sEpi + ew * epi_warp_bytes(EPI));
+    const uint32_t st_f32 = stage_base;
+    const uint32_t st_out0 = stage_base + (EPI == EPI_BIAS_GELU ? EPI_F32_TILE : 0);
+    const uint32_t st_out1 = st_out0 + EPI_BF16_TILE;
     uint32_t tempty_addr[2] = {0u, 0u};
     if constexpr (PAIR) {
 #pragma unroll
@@ -528,9 +546,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int mb, nb;
       tile_coords(tile, p, mb, nb);
       const int row_block = mb * Cfg::CTAS + static_cast<int>(rank);  // this CTA's 128-row block
-      const int row = row_block * BM + q * 32 + lane;
+      const int row0 = row_block * BM + q * 32;  // this warp's first row
+      const int row = row0 + lane;
       const bool row_ok = row < p.M;
-      const size_t row_off = static_cast<size_t>(row) * static_cast<size_t>(p.N);
       float sum[EPI == EPI_SHARD_SUM ? 128 : 1];
       for (int s = 0; s < p.shards; ++s, ++unit) {
         const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
@@ -548,6 +566,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (col >= p.N) continue;  // warp-uniform: ragged last column block
           uint32_t r[32];
           tmem_load_32cols(t_addr + c * 32, r);
+          // the staging tiles are free again once this warp's previous bulk
+          // stores have read them
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
           if constexpr (EPI == EPI_BIAS_GELU) {
             // Z = X·A + a (fp32, saved), H = g(Z) saved as (hi, lo)
             float bias[32];
@@ -558,16 +580,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(r[j]) + bias[j];
 #pragma unroll
             for (int j = 0; j < 16; ++j) split_bf16x2(gelu_f(z[2 * j]), gelu_f(z[2 * j + 1]), hp[j], lp[j]);
-            if (row_ok) {
-              store_f32x32(p.out_f32 + row_off + col, z);
-              store_bf16x32(p.out0 + row_off + col, hp);
-              store_bf16x32(p.out1 + row_off + col, lp);
+            stage_f32x32(st_f32, lane, z);
+            stage_bf16x32(st_out0, lane, hp);
+            stage_bf16x32(st_out1, lane, lp);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out[2], st_f32, col, row0);
+              tma_store_2d(&maps.out[0], st_out0, col, row0);
+              tma_store_2d(&maps.out[1], st_out1, col, row0);
+              bulk_commit_group();
             }
           } else if constexpr (EPI == EPI_GELU_GRAD) {
             // dH = (dY·Bᵀ) ⊙ g'(Z), saved as (hi, lo); fp32 column sums for da
             float z[32];
             if (row_ok) {
-              load_f32x32(p.aux + row_off + col, z);
+              load_f32x32(p.aux + static_cast<size_t>(row) * static_cast<size_t>(p.N) + col, z);
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j) z[j] = 0.0f;
@@ -578,9 +606,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t hp[16], lp[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) split_bf16x2(dh[2 * j], dh[2 * j + 1], hp[j], lp[j]);
-            if (row_ok) {
-              store_bf16x32(p.out0 + row_off + col, hp);
-              store_bf16x32(p.out1 + row_off + col, lp);
+            stage_bf16x32(st_out0, lane, hp);
+            stage_bf16x32(st_out1, lane, lp);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out[0], st_out0, col, row0);
+              tma_store_2d(&maps.out[1], st_out1, col, row0);
+              bulk_commit_group();
             }
             if (p.colsum != nullptr) {
               const float cs = warp_column_sums(dh);
@@ -590,7 +623,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t op[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) op[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-            if (row_ok) store_bf16x32(p.out0 + row_off + col, op);
+            stage_bf16x32(st_out0, lane, op);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out[0], st_out0, col, row0);
+              bulk_commit_group();
+            }
           } else {  // EPI_SHARD_SUM
             if (s == 0) {
 #pragma unroll
@@ -611,7 +650,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j)
                 yp[j] = pack_bf16x2(sum[c * 32 + 2 * j] + bias[2 * j], sum[c * 32 + 2 * j + 1] + bias[2 * j + 1]);
-              if (row_ok) store_bf16x32(p.out0 + row_off + col, yp);
+              stage_bf16x32(st_out0, lane, yp);
+              fence_proxy_async_shared();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&maps.out[0], st_out0, col, row0);
+                bulk_commit_group();
+              }
             }
           }
         }
@@ -626,6 +671,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
+    // every bulk store this warp issued has completed before the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // Both CTAs of a pair stay resident until all remote arrivals and

@@ -81,7 +81,7 @@ constexpr bool kPair = MLPTP_USE_PAIR != 0;
 #define MLPTP_WIDE_TN 512
 #endif
 constexpr int kWideTN = kPair ? MLPTP_WIDE_TN : 256;
-using TileShape = TileCfg<kPair>;
+using TileShape = TileCfg<kPair, 256, EPI_STORE>;
 // 128-row blocks that a GEMM over R rows covers (whole tiles).
 size_t gemm_row_blocks(int64_t R) {
   return static_cast<size_t>((R + TileShape::TILE_M - 1) / TileShape::TILE_M) * TileShape::CTAS;
@@ -194,6 +194,26 @@ mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t c
   return MLP_OK;
 }
 
+// Output of a GEMM epilogue: row-major [rows, cols], stored in 32x32 boxes
+// from the epilogue's swizzled staging tiles (bf16: 64-byte swizzle, fp32:
+// 128-byte swizzle, matching the staging layout in gemm.cuh).
+mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, bool f32, const char* name) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t esz = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esz};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for output of %s (CUresult %d)", name, (int)r);
+  return MLP_OK;
+}
+
 // Operand of the GEMM: `rows` is its M (or N) extent, `k` its K extent.
 // K-major: stored [rows, k];  MN-major: stored [k, rows].
 mlp_status_t make_operand_map(CUtensorMap* map, const void* ptr, bool mn_major, int64_t rows, int64_t k,
@@ -227,7 +247,7 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
 // template instance).
 template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN>
 mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
-  using Cfg = TileCfg<PAIR, TN>;
+  using Cfg = TileCfg<PAIR, TN, EPI>;
   static std::mutex mu;
   static uint64_t done_mask = 0;
   static int clusters[64] = {};
@@ -269,9 +289,16 @@ struct Launch {
 
 template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
-  using Cfg = TileCfg<PAIR, TN>;
+  using Cfg = TileCfg<PAIR, TN, EPI>;
   if (g.M == 0 || g.N == 0) return MLP_OK;
   GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  {
+    mlp_status_t st = make_out_map(&maps.out[0], p.out0, g.M, g.N, false, name);
+    if (st == MLP_OK && p.out1 != nullptr) st = make_out_map(&maps.out[1], p.out1, g.M, g.N, false, name);
+    if (st == MLP_OK && p.out_f32 != nullptr) st = make_out_map(&maps.out[2], p.out_f32, g.M, g.N, true, name);
+    if (st != MLP_OK) return st;
+  }
   for (int i = 0; i < 2; ++i) {
     mlp_status_t st = make_operand_map(&maps.a[i], g.a.p[i], A_MN, g.M, g.K, BM, name);
     if (st != MLP_OK) return st;
