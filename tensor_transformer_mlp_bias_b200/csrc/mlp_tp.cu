@@ -71,16 +71,26 @@ size_t colsum_chunks(int64_t R) { return static_cast<size_t>((R + COLSUM_ROWS_PE
 #define MLPTP_USE_PAIR 1
 #endif
 constexpr bool kPair = MLPTP_USE_PAIR != 0;
-// Column tile of the weight-gradient GEMMs: 512 (two MMA widths per CTA
-// pair, one TMEM accumulator) reads 25% fewer operand bytes per FLOP from
-// L2, which bounds these GEMMs.  GEMMs with a heavy epilogue (bias+GeLU with
-// three outputs, GeLU derivative with two outputs and column sums) and the
-// shard-sum GEMMs keep 256 columns and two accumulators, so the epilogue of
-// one tile overlaps the mainloop of the next.
+// Column tiles.  512 (two MMA widths per CTA pair, one TMEM accumulator)
+// reads 25% fewer operand bytes per FLOP from L2, which bounds these GEMMs;
+// 256 keeps two accumulators so the epilogue of one tile overlaps the
+// mainloop of the next.  Measured on B200: 512 for the weight gradients and
+// the bias+GeLU GEMM (its outputs leave through asynchronous TMA stores);
+// 256 for the GeLU-derivative GEMM (its epilogue waits on loads of Z) and
+// for the shard-sum GEMMs (the running sum of the shard partials is held in
+// registers, 128 values per thread at 256 columns).
 #ifndef MLPTP_WIDE_TN
 #define MLPTP_WIDE_TN 512
 #endif
 constexpr int kWideTN = kPair ? MLPTP_WIDE_TN : 256;
+#ifndef MLPTP_FC1_TN
+#define MLPTP_FC1_TN 512
+#endif
+#ifndef MLPTP_FC2BD_TN
+#define MLPTP_FC2BD_TN 256
+#endif
+constexpr int kFc1TN = kPair ? MLPTP_FC1_TN : 256;    // bias+GeLU GEMM
+constexpr int kFc2BdTN = kPair ? MLPTP_FC2BD_TN : 256;  // GeLU-derivative GEMM
 using TileShape = TileCfg<kPair, 256, EPI_STORE>;
 // 128-row blocks that a GEMM over R rows covers (whole tiles).
 size_t gemm_row_blocks(int64_t R) {
@@ -396,7 +406,7 @@ mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const voi
   p.out1 = static_cast<__nv_bfloat16*>(H_lo);
   p.bias = static_cast<const __nv_bfloat16*>(a);
   GemmDesc g{one(X, false), one(A, true), s.T, s.f, s.h, 1, 1};
-  return launch_gemm<false, true, EPI_BIAS_GELU>(g, p, L, "column-parallel forward (Z, H)");
+  return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H)");
 }
 
 mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const void* B, const void* b, void* Y,
@@ -418,7 +428,7 @@ mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, co
   p.aux = static_cast<const float*>(Z);
   p.colsum = da != nullptr ? partials(ws, s) : nullptr;
   GemmDesc g{one(dY, false), one(B, false), s.T, s.f, s.h, 1, 1};
-  mlp_status_t st = launch_gemm<false, false, EPI_GELU_GRAD>(g, p, L, "row-parallel backward data (dH, da)");
+  mlp_status_t st = launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN>(g, p, L, "row-parallel backward data (dH, da)");
   if (st != MLP_OK || da == nullptr) return st;
   return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream);
 }
