@@ -168,6 +168,33 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
                                         void* dA,
                                         void* ws, size_t ws_bytes, void* stream);
 
+/* ----------------------------------------------------- recomputation */
+
+/* Activation recomputation ("Megatron-LM（英伟达超大模型训练框架）完整介绍", §三
+ * 显存优化关键技术, item 2 激活重计算: drop the intermediate activations and
+ * recompute them in the backward; "Megatron-LM 深度解读报告" §二 2.7 table).
+ * mlp_tp_forward_recompute keeps Z, H and H_lo only in the workspace, where
+ * the next call may overwrite them, so nothing of size T·f outlives the
+ * forward; mlp_tp_backward_recompute reruns the column-parallel GEMM from X
+ * (one extra 2·T·h·f product, bit-identical Z, H, H_lo) and then runs the
+ * backward of mlp_tp_backward.  Both need
+ * mlp_tp_recompute_workspace_bytes(T, h, f, t) bytes of workspace (the
+ * ordinary workspace plus T·f·8 bytes for Z, H, H_lo).  Same conventions
+ * and split flags as mlp_tp_forward / mlp_tp_backward. */
+size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
+
+mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* a,
+                                      const void* B, const void* b,
+                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                                      void* Y,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void* A,
+                                       const void* a, const void* B,
+                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                                       void* dX, void* dA, void* da, void* dB, void* db,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------- allocation-free */
 
 /* db = sum over rows of dY (the row-parallel layer's bias gradient, as

@@ -42,6 +42,10 @@ _SIGS = {
     "mlp_tp_fc2_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_fc1_backward_data": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_fc1_backward_weight": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_recompute_workspace_bytes": ([_I64, _I64, _I64, _I32], _SZ),
+    "mlp_tp_forward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_backward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 5 + [_P, _SZ, _P],
+                                  ctypes.c_int),
     "mlp_tp_fc2_bias_grad_noalloc": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "mlp_tp_check": ([_P, _P], ctypes.c_int),
     "mlp_tp_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -194,6 +198,33 @@ def mlp_tp_fc1_backward_weight(X, dH, dH_lo, T, h, f, t, dA, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_fc1_backward_weight(_addr(X, "X"), _addr(dH, "dH"), _addr(dH_lo, "dH_lo"), T, h, f, t,
                                             _addr(dA, "dA"), w, wn, _stream(stream)))
+
+
+def recompute_workspace_bytes(T: int, h: int, f: int, t: int) -> int:
+    return int(lib().mlp_tp_recompute_workspace_bytes(T, h, f, t))
+
+
+def make_recompute_workspace(T: int, h: int, f: int, t: int, device="cuda"):
+    import torch
+    n = recompute_workspace_bytes(T, h, f, t)
+    if n == 0:
+        raise MlpError(2, f"unsupported shape T={T} h={h} f={f} t={t}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def mlp_tp_forward_recompute(X, A, a, B, b, T, h, f, t, split, Y, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_forward_recompute(_addr(X, "X", T == 0), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"),
+                                          _addr(b, "b"), T, h, f, t, split, _addr(Y, "Y", T == 0), w, wn,
+                                          _stream(stream)))
+
+
+def mlp_tp_backward_recompute(dY, X, A, a, B, T, h, f, t, split, dX, dA, da, dB, db, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_backward_recompute(_addr(dY, "dY", T == 0), _addr(X, "X", T == 0), _addr(A, "A"),
+                                           _addr(a, "a"), _addr(B, "B"), T, h, f, t, split,
+                                           _addr(dX, "dX", T == 0), _addr(dA, "dA"), _addr(da, "da", True),
+                                           _addr(dB, "dB"), _addr(db, "db", True), w, wn, _stream(stream)))
 
 
 def mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db, stream=None):

@@ -110,6 +110,15 @@ size_t workspace_bytes(const Shape& s) {
   return partial_offset(s) + align_up((da_rows > db_rows ? da_rows : db_rows) * sizeof(float), 256);
 }
 
+// Recomputation keeps Z, H and H_lo in the workspace after the rest:
+// [ ... | Z fp32 | H | H_lo ].
+size_t recompute_z_offset(const Shape& s) { return workspace_bytes(s); }
+size_t recompute_h_offset(const Shape& s) {
+  return recompute_z_offset(s) + align_up(static_cast<size_t>(s.T * s.f * 4), 256);
+}
+size_t recompute_hlo_offset(const Shape& s) { return recompute_h_offset(s) + pair_bytes(s); }
+size_t recompute_workspace_bytes(const Shape& s) { return recompute_hlo_offset(s) + pair_bytes(s); }
+
 struct Ptr {
   const void* p;
   const char* name;
@@ -129,10 +138,10 @@ mlp_status_t check_ptrs(std::initializer_list<Ptr> ptrs) {
   return MLP_OK;
 }
 
-mlp_status_t check_ws(const Shape& s, void* ws, size_t ws_bytes) {
+mlp_status_t check_ws(const Shape& s, void* ws, size_t ws_bytes, bool recompute = false) {
   if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MLP_ERR_MISALIGNED, "workspace is not 256-byte aligned");
-  const size_t need = workspace_bytes(s);
+  const size_t need = recompute ? recompute_workspace_bytes(s) : workspace_bytes(s);
   if (ws_bytes < need)
     return fail(MLP_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
   return MLP_OK;
@@ -467,12 +476,12 @@ mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, 
 
 // Common preamble: shape, pointers, workspace, device.
 mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, void* stream,
-                      Launch& L) {
+                      Launch& L, bool recompute = false) {
   mlp_status_t st = check_shape(s);
   if (st != MLP_OK) return st;
   st = check_ptrs(ptrs);
   if (st != MLP_OK) return st;
-  st = check_ws(s, ws, ws_bytes);
+  st = check_ws(s, ws, ws_bytes, recompute);
   if (st != MLP_OK) return st;
   L.stream = static_cast<cudaStream_t>(stream);
   return current_device(L.dev, L.sms);
@@ -592,6 +601,61 @@ mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const
   if (st != MLP_OK) return st;
   void* dH = static_cast<char*>(ws) + dh_offset();
   void* dH_lo = static_cast<char*>(ws) + dh_lo_offset(s);
+  if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
+  if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
+  if ((st = fc1_backward_data(s, dH, (split & MLP_TP_SPLIT_FC1_BACKWARD_DATA) ? dH_lo : nullptr, A, dX, ws, L)) !=
+      MLP_OK)
+    return st;
+  return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
+}
+
+size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t) {
+  Shape s{T, h, f, t};
+  std::string saved = g_last_error;
+  const bool ok = check_shape(s) == MLP_OK;
+  g_last_error = saved;
+  return ok ? recompute_workspace_bytes(s) : 0;
+}
+
+mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* a, const void* B, const void* b,
+                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* Y, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = check_split(split);
+  if (st != MLP_OK) return st;
+  st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
+                    {Y, "Y", false, s.T == 0}},
+                ws, ws_bytes, stream, L, true);
+  if (st != MLP_OK) return st;
+  char* w = static_cast<char*>(ws);
+  void* Z = w + recompute_z_offset(s);
+  void* H = w + recompute_h_offset(s);
+  void* H_lo = w + recompute_hlo_offset(s);
+  if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
+  return fc2_forward(s, H, (split & MLP_TP_SPLIT_FC2_FORWARD) ? H_lo : nullptr, B, b, Y, ws, L);
+}
+
+mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void* A, const void* a, const void* B,
+                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* dX, void* dA,
+                                       void* da, void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = check_split(split);
+  if (st != MLP_OK) return st;
+  st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false},
+                    {B, "B", false}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
+                    {dB, "dB", false}, {db, "db", true}},
+                ws, ws_bytes, stream, L, true);
+  if (st != MLP_OK) return st;
+  char* w = static_cast<char*>(ws);
+  void* Z = w + recompute_z_offset(s);
+  void* H = w + recompute_h_offset(s);
+  void* H_lo = w + recompute_hlo_offset(s);
+  void* dH = w + dh_offset();
+  void* dH_lo = w + dh_lo_offset(s);
+  // recompute the activations the forward did not keep, then the backward
+  if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
   if ((st = fc1_backward_data(s, dH, (split & MLP_TP_SPLIT_FC1_BACKWARD_DATA) ? dH_lo : nullptr, A, dX, ws, L)) !=

@@ -50,6 +50,15 @@ def test_workspace_bytes(lib):
     assert binding.workspace_bytes(-1, 256, 1024, 2) == 0
 
 
+def test_recompute_workspace_bytes(lib):
+    T, h, f, t = 200, 192, 384, 6
+    base = binding.workspace_bytes(T, h, f, t)
+    rnd = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    # the ordinary workspace, then Z (fp32) and the H pair
+    assert binding.recompute_workspace_bytes(T, h, f, t) == base + rnd(T * f * 4) + 2 * rnd(T * f * 2)
+    assert binding.recompute_workspace_bytes(T, h, 100, t) == 0
+
+
 FAKE = 1 << 20  # a 16-byte aligned fake address: validation must fail before any use
 
 
