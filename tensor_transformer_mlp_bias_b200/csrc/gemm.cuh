@@ -354,6 +354,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
   }
   tc_fence_after_sync();
+  // Everything above touches only this CTA's shared memory, TMEM and the
+  // kernel parameters, so it may overlap the previous kernel's tail; every
+  // global read and write below comes after the previous grid completed.
+  grid_launch_dependents();
+  grid_wait_prerequisites();
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
   const uint64_t budget = p.budget_ns;

@@ -346,17 +346,19 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
   const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = Cfg::CTAS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see grid_wait_prerequisites
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = Cfg::CTAS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CTAS));
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = L.stream;
   cfg.attrs = attr;
-  cfg.numAttrs = PAIR ? 1 : 0;
+  cfg.numAttrs = PAIR ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN>, maps, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);

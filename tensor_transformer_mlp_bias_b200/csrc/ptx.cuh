@@ -283,3 +283,17 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 }  // namespace mlptp
+
+// ------------------------------------------------------------------ dependent launch
+namespace mlptp {
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue on SMs this grid frees, and wait (here) until the previous grid
+// in the stream has completed and its memory is visible.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace mlptp
