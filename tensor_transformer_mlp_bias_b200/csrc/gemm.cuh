@@ -116,6 +116,11 @@ constexpr unsigned int STATUS_TIMEOUT = 7u;
 struct GemmParams {
   int M, N;
   int shards;             // K segments reduced in the epilogue (EPI_SHARD_SUM); 1 otherwise
+  // Work list: tiles [0, full_tiles) whole; each later tile (the partial last
+  // wave) as tail_split pieces of shards/tail_split consecutive shards whose
+  // fp32 sums go to tail_scratch (a separate kernel adds the pieces).
+  int full_tiles, tail_split, num_work;
+  float* tail_scratch;    // [pieces][TILE_M][BN] fp32
   int parts;              // 1, or 2 when an operand is a bf16 (hi, lo) pair
   int kblocks_per_shard;  // BK-wide K slices per segment and part
   int m_blocks, n_blocks, num_tiles, group_m;
@@ -163,6 +168,20 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
   const int r = tile - g * per_group;
   mb = first_m + r % gsz;
   nb = r / gsz;
+}
+
+// One item of the work list: a whole tile (piece < 0, shards [0, shards)) or
+// one piece of a split tile (shards [s_begin, s_end)).
+struct WorkItem {
+  int tile, s_begin, s_end, piece;
+};
+
+__device__ __forceinline__ WorkItem work_item(int w, const GemmParams& p) {
+  if (w < p.full_tiles) return WorkItem{w, 0, p.shards, -1};
+  const int piece = w - p.full_tiles;
+  const int per = p.shards / p.tail_split;
+  const int part = piece % p.tail_split;
+  return WorkItem{p.full_tiles + piece / p.tail_split, part * per, part * per + per, piece};
 }
 
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort, unsigned int where) {
@@ -372,13 +391,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage: armed at least once / parity of last arming
       bool ok = true;
       bool first = true;
-      for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
+      for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
+        const WorkItem it = work_item(w, p);
         int mb, nb;
-        tile_coords(tile, p, mb, nb);
+        tile_coords(it.tile, p, mb, nb);
         const int m0 = mb * Cfg::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
         // this CTA's B rows for MMA width w start at n0 + w * BN
         const int n0 = nb * Cfg::TILE_N + static_cast<int>(rank) * Cfg::SUB_ROWS;
-        for (int s = 0; ok && s < p.shards; ++s) {
+        for (int s = it.s_begin; ok && s < it.s_end; ++s) {
           for (int i = 0; i < kb_per_unit; ++i) {
             if ((p.debug_flags & 1u) && !first) {
               ok = false;  // test hook: stop feeding the tensor core after one stage
@@ -463,8 +483,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, unit = 0;
       bool ok = true;
-      for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
-        for (int s = 0; ok && s < p.shards; ++s, ++unit) {
+      for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
+        const WorkItem it = work_item(w, p);
+        for (int s = it.s_begin; ok && s < it.s_end; ++s, ++unit) {
           const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
           if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, abort_flag, budget)) {
             record_timeout(p, abort_flag, 0x200u);
@@ -547,15 +568,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     uint32_t unit = 0;
     bool ok = true;
-    for (int tile = cluster_id; ok && tile < p.num_tiles; tile += num_clusters) {
+    for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
+      const WorkItem it = work_item(w, p);
       int mb, nb;
-      tile_coords(tile, p, mb, nb);
+      tile_coords(it.tile, p, mb, nb);
       const int row_block = mb * Cfg::CTAS + static_cast<int>(rank);  // this CTA's 128-row block
       const int row0 = row_block * BM + q * 32;  // this warp's first row
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
       float sum[EPI == EPI_SHARD_SUM ? 128 : 1];
-      for (int s = 0; s < p.shards; ++s, ++unit) {
+      for (int s = it.s_begin; s < it.s_end; ++s, ++unit) {
         const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
         if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort_flag, budget)) {
           record_timeout(p, abort_flag, 0x400u);
@@ -636,14 +658,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               bulk_commit_group();
             }
           } else {  // EPI_SHARD_SUM
-            if (s == 0) {
+            if (s == it.s_begin) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) sum[c * 32 + j] = __uint_as_float(r[j]);
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j) sum[c * 32 + j] += __uint_as_float(r[j]);
             }
-            if (s == p.shards - 1) {
+            if (s == it.s_end - 1 && it.piece >= 0) {
+              // one piece of a split tile: its fp32 sum goes to the scratch
+              float* dst = p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * BN) +
+                           static_cast<size_t>(rank * BM + q * 32 + lane) * BN + half * 128 + c * 32;
+              float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(sum[c * 32 + 4 * j], sum[c * 32 + 4 * j + 1], sum[c * 32 + 4 * j + 2],
+                                    sum[c * 32 + 4 * j + 3]);
+            } else if (s == it.s_end - 1) {
               float bias[32];
               if (p.bias != nullptr) {
                 load_bf16x32(p.bias + col, bias);
@@ -698,6 +729,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_dealloc(tmem_base, TMEM_COLS);
     }
   }
+}
+
+// Finishes the split tiles of a shard-sum GEMM: out[row, col] = bf16(
+// ((piece_0 + piece_1) + ...) + bias[col]), pieces in ascending shard order.
+// One thread per 8 consecutive columns of one row of one split tile.
+template <int TILE_M>
+__global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmParams p) {
+  constexpr int COLS8 = BN / 8;
+  const int tail_tiles = (p.num_work - p.full_tiles) / p.tail_split;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(tail_tiles) * TILE_M * COLS8) return;
+  const int t_local = static_cast<int>(idx / (TILE_M * COLS8));
+  const int rem = static_cast<int>(idx % (TILE_M * COLS8));
+  const int r = rem / COLS8, c8 = (rem % COLS8) * 8;
+  int mb, nb;
+  tile_coords(p.full_tiles + t_local, p, mb, nb);
+  const int row = mb * TILE_M + r, col = nb * BN + c8;
+  if (row >= p.M || col >= p.N) return;
+  float acc[8];
+  for (int part = 0; part < p.tail_split; ++part) {
+    const float4* src = reinterpret_cast<const float4*>(
+        p.tail_scratch + static_cast<size_t>(t_local * p.tail_split + part) * (TILE_M * BN) +
+        static_cast<size_t>(r) * BN + c8);
+    const float4 v0 = src[0], v1 = src[1];
+    const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = part == 0 ? v[e] : acc[e] + v[e];
+  }
+  float bias[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) bias[e] = 0.0f;
+  if (p.bias != nullptr) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(u[e]);
+      bias[2 * e] = f.x;
+      bias[2 * e + 1] = f.y;
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0] + bias[0], acc[1] + bias[1]);
+  o.y = pack_bf16x2(acc[2] + bias[2], acc[3] + bias[3]);
+  o.z = pack_bf16x2(acc[4] + bias[4], acc[5] + bias[5]);
+  o.w = pack_bf16x2(acc[6] + bias[6], acc[7] + bias[7]);
+  *reinterpret_cast<uint4*>(p.out0 + static_cast<size_t>(row) * p.N + col) = o;
 }
 
 }  // namespace mlptp

@@ -102,13 +102,25 @@ size_t pair_bytes(const Shape& s) { return align_up(static_cast<size_t>(s.T * s.
 size_t dh_offset() { return WS_HEADER_BYTES; }
 size_t dh_lo_offset(const Shape& s) { return WS_HEADER_BYTES + pair_bytes(s); }
 size_t partial_offset(const Shape& s) { return WS_HEADER_BYTES + 2 * pair_bytes(s); }
-size_t workspace_bytes(const Shape& s) {
+size_t partial_bytes(const Shape& s) {
   // da: one row of column sums per (128-row block, 32-row lane quadrant);
   // db: one row per COLSUM_ROWS_PER_CHUNK rows of dY.
   const size_t da_rows = gemm_row_blocks(s.T) * 4 * static_cast<size_t>(s.f);
   const size_t db_rows = colsum_chunks(s.T) * static_cast<size_t>(s.h);
-  return partial_offset(s) + align_up((da_rows > db_rows ? da_rows : db_rows) * sizeof(float), 256);
+  return align_up((da_rows > db_rows ? da_rows : db_rows) * sizeof(float), 256);
 }
+// Pieces of split tiles of the shard-sum GEMMs (outputs [T, h]): at most
+// one piece per shard of every tile, and at most TAIL_MAX_PIECES.
+constexpr size_t TAIL_MAX_PIECES = 256;
+constexpr size_t TAIL_PIECE_BYTES = static_cast<size_t>(TileShape::TILE_M) * BN * sizeof(float);
+size_t tail_pieces_capacity(const Shape& s) {
+  const size_t tiles = static_cast<size_t>((s.T + TileShape::TILE_M - 1) / TileShape::TILE_M) *
+                       static_cast<size_t>((s.h + BN - 1) / BN);
+  const size_t n = tiles * static_cast<size_t>(s.t);
+  return n < TAIL_MAX_PIECES ? n : TAIL_MAX_PIECES;
+}
+size_t tail_offset(const Shape& s) { return partial_offset(s) + partial_bytes(s); }
+size_t workspace_bytes(const Shape& s) { return tail_offset(s) + tail_pieces_capacity(s) * TAIL_PIECE_BYTES; }
 
 // Recomputation keeps Z, H and H_lo in the workspace after the rest:
 // [ ... | Z fp32 | H | H_lo ].
@@ -252,6 +264,8 @@ struct GemmDesc {
   int64_t M, N, K;  // K = shards * (K of one shard); each part spans all of K
   int shards;
   int parts;
+  float* tail_scratch = nullptr;  // shard-sum GEMMs: room for split pieces of the last wave
+  size_t tail_capacity = 0;       // pieces
 };
 
 // Tile order.  All resident tiles walk K in near lockstep, so DRAM traffic
@@ -344,7 +358,34 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN>(L.dev, L.sms, &max_clusters);
   if (st != MLP_OK) return st;
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
-  const int clusters = p.num_tiles < max_clusters ? p.num_tiles : max_clusters;
+  // Work list.  A shard-sum GEMM whose last wave is partial splits each tile
+  // of that wave into k pieces of shards/k consecutive shards, k a divisor of
+  // the shard count chosen to minimise the time of that wave,
+  // ceil(tail*k/clusters)/k tiles, within the scratch capacity.
+  p.full_tiles = p.num_tiles;
+  p.tail_split = 1;
+  if (EPI == EPI_SHARD_SUM && p.shards > 1 && g.tail_scratch != nullptr) {
+    const int tail = p.num_tiles % max_clusters;
+    if (tail > 0) {
+      int best_k = 1;
+      double best = 1.0;
+      for (int k = 2; k <= p.shards; ++k) {
+        if (p.shards % k != 0 || static_cast<size_t>(tail) * k > g.tail_capacity) continue;
+        const double cost = static_cast<double>((tail * k + max_clusters - 1) / max_clusters) / k;
+        if (cost < best - 1e-9) {
+          best = cost;
+          best_k = k;
+        }
+      }
+      if (best_k > 1) {
+        p.full_tiles = p.num_tiles - tail;
+        p.tail_split = best_k;
+        p.tail_scratch = g.tail_scratch;
+      }
+    }
+  }
+  p.num_work = p.full_tiles + (p.num_tiles - p.full_tiles) * p.tail_split;
+  const int clusters = p.num_work < max_clusters ? p.num_work : max_clusters;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see grid_wait_prerequisites
@@ -363,6 +404,13 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
+  if (p.tail_split > 1) {
+    const long long threads = static_cast<long long>(p.num_tiles - p.full_tiles) * Cfg::TILE_M * (BN / 8);
+    tail_reduce_kernel<Cfg::TILE_M><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, L.stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "tail_reduce");
+    g_launches.fetch_add(1);
+  }
   return MLP_OK;
 }
 
@@ -407,6 +455,9 @@ Operand pair(const void* hi, const void* lo, bool mn) { return Operand{{hi, lo !
 float* partials(void* ws, const Shape& s) {
   return reinterpret_cast<float*>(static_cast<char*>(ws) + partial_offset(s));
 }
+float* tail_scratch(void* ws, const Shape& s) {
+  return reinterpret_cast<float*>(static_cast<char*>(ws) + tail_offset(s));
+}
 
 // ---------------------------------------------------------------- stages
 mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H, void* H_lo,
@@ -425,7 +476,8 @@ mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const 
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(Y);
   p.bias = static_cast<const __nv_bfloat16*>(b);
-  GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, s.t, H_lo != nullptr ? 2 : 1};
+  GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, s.t, H_lo != nullptr ? 2 : 1,
+             tail_scratch(ws, s), tail_pieces_capacity(s)};
   return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, L, "row-parallel forward + shard reduce (Y)");
 }
 
@@ -463,7 +515,8 @@ mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* dH_lo
                                const Launch& L) {
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dX);
-  GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, s.t, dH_lo != nullptr ? 2 : 1};
+  GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, s.t, dH_lo != nullptr ? 2 : 1,
+             tail_scratch(ws, s), tail_pieces_capacity(s)};
   return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, L, "column-parallel backward data + shard reduce (dX)");
 }
 

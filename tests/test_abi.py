@@ -41,9 +41,10 @@ def test_status_strings(lib):
 
 def test_workspace_bytes(lib):
     n = binding.workspace_bytes(64, 256, 1024, 2)
-    # header 256 + dH pair 2*64*1024*2 + da partials: one 256-row pair tile = two 128-row blocks,
-    # 4 lane quadrants each, f fp32 column sums per quadrant
-    assert n == 256 + 2 * 64 * 1024 * 2 + 2 * 4 * 1024 * 4
+    # header 256 + dH pair 2*64*1024*2 + da partials (one 256-row pair tile = two 128-row blocks,
+    # 4 lane quadrants each, f fp32 column sums per quadrant) + room for the split pieces of the
+    # shard-sum GEMMs' last wave (1 tile x t=2 shards, 256x256 fp32 each)
+    assert n == 256 + 2 * 64 * 1024 * 2 + 2 * 4 * 1024 * 4 + 2 * 256 * 256 * 4
     assert binding.workspace_bytes(64, 256, 1000, 2) == 0   # f/t not a multiple of 64
     assert binding.workspace_bytes(64, 100, 1024, 2) == 0   # h not a multiple of 64
     assert binding.workspace_bytes(64, 256, 1024, 0) == 0   # t < 1
