@@ -229,6 +229,7 @@ def main():
                     help="split flags: 1 = Y from the (H, H_lo) pair, 2 = dX from the (dH, dH_lo) pair")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-t", action="store_true", help="time only the headline shard count")
     ap.add_argument("--clock-interval-ms", type=int, default=100,
                     help="nvidia-smi sampling period during the timed region")
     args = ap.parse_args()
@@ -311,6 +312,40 @@ def main():
     max_ms, total_flops = reduce_max_sum(local_ms, float(wl.flops) * args.steps)
     value = total_flops / (max_ms * 1e-3) / 1e12
     ms_per_step = max_ms / args.steps
+
+    # ------------------------------------------------ the workload's other shard counts
+    # Same device-resident step (stage calls) for every other t the workload
+    # lists, on the same inputs; reported beside the headline t.
+    per_t = {}
+    for t_other in wl.shards:
+        if t_other == t or args.no_per_t:
+            continue
+        ws_o = binding.make_workspace(T, h, f, t_other)
+
+        def step_o():
+            binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t_other, Z, H, H_lo, ws_o, sh)
+            binding.mlp_tp_fc2_forward(H, H_lo2, dev["B"], dev["b"], T, h, f, t_other, Y, ws_o, sh)
+            binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t_other, dH, dH_lo, da, ws_o, sh)
+            binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t_other, dB, db, ws_o, sh)
+            binding.mlp_tp_fc1_backward_data(dH, dH_lo2, dev["A"], T, h, f, t_other, dX, ws_o, sh)
+            binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t_other, dA, ws_o, sh)
+
+        for _ in range(3):
+            step_o()
+        n_o = max(10, args.steps // 4)
+        s_o, e_o = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        s_o.record(stream)
+        for _ in range(n_o):
+            step_o()
+        e_o.record(stream)
+        torch.cuda.synchronize()
+        binding.mlp_tp_check(ws_o, sh)
+        ms_o, fl_o = reduce_max_sum(s_o.elapsed_time(e_o), float(wl.flops) * n_o)
+        per_t[str(t_other)] = {"value": fl_o / (ms_o * 1e-3) / 1e12, "ms_per_step": ms_o / n_o, "steps": n_o}
+        del ws_o
+    per_t[str(t)] = {"value": value, "ms_per_step": ms_per_step, "steps": args.steps}
 
     # ------------------------------------------------ end-to-end through the public API
     # Each step copies its inputs from pinned host memory, runs mlp_tp_forward
@@ -417,6 +452,7 @@ def main():
         "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_DENSE_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * value / world / float(peaks.get("bf16_tflops", 1713.1)),
         "stage_ms": stage_ms,
+        "per_t": dict(sorted(per_t.items(), key=lambda kv: int(kv[0]))),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps,
