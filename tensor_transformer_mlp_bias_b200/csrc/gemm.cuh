@@ -116,11 +116,14 @@ constexpr unsigned int STATUS_TIMEOUT = 7u;
 struct GemmParams {
   int M, N;
   int shards;             // K segments reduced in the epilogue (EPI_SHARD_SUM); 1 otherwise
-  // Work list: tiles [0, full_tiles) whole; each later tile (the partial last
-  // wave) as tail_split pieces of shards/tail_split consecutive shards whose
-  // fp32 sums go to tail_scratch (a separate kernel adds the pieces).
-  int full_tiles, tail_split, num_work;
-  float* tail_scratch;    // [pieces][TILE_M][BN] fp32
+  // Work list.  Without a K split: tiles [0, full_tiles) whole; each later
+  // tile (the partial last wave of a shard-sum GEMM) as tail_split pieces of
+  // shards/tail_split consecutive shards.  With a K split (kb_split > 1, GEMMs
+  // without shards and with fewer tiles than CTA pairs): every tile as
+  // kb_split pieces of consecutive K slices.  A piece's fp32 sum goes to
+  // tail_scratch and a separate kernel adds the pieces of a tile in order.
+  int full_tiles, tail_split, kb_split, num_work;
+  float* tail_scratch;    // [pieces][TILE_M][TILE_N] fp32
   int parts;              // 1, or 2 when an operand is a bf16 (hi, lo) pair
   int kblocks_per_shard;  // BK-wide K slices per segment and part
   int m_blocks, n_blocks, num_tiles, group_m;
@@ -170,18 +173,24 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
   nb = r / gsz;
 }
 
-// One item of the work list: a whole tile (piece < 0, shards [0, shards)) or
-// one piece of a split tile (shards [s_begin, s_end)).
+// One item of the work list: a whole tile (piece < 0) or one piece of a
+// split tile: shards [s_begin, s_end) and, within each shard, the K slices
+// [i_begin, i_end) of the parts x K-blocks loop.
 struct WorkItem {
-  int tile, s_begin, s_end, piece;
+  int tile, s_begin, s_end, i_begin, i_end, piece;
 };
 
-__device__ __forceinline__ WorkItem work_item(int w, const GemmParams& p) {
-  if (w < p.full_tiles) return WorkItem{w, 0, p.shards, -1};
+__device__ __forceinline__ WorkItem work_item(int w, const GemmParams& p, int kb_per_unit) {
+  if (p.kb_split > 1) {
+    const int chunk = w % p.kb_split;
+    return WorkItem{w / p.kb_split, 0, p.shards, chunk * kb_per_unit / p.kb_split,
+                    (chunk + 1) * kb_per_unit / p.kb_split, w};
+  }
+  if (w < p.full_tiles) return WorkItem{w, 0, p.shards, 0, kb_per_unit, -1};
   const int piece = w - p.full_tiles;
   const int per = p.shards / p.tail_split;
   const int part = piece % p.tail_split;
-  return WorkItem{p.full_tiles + piece / p.tail_split, part * per, part * per + per, piece};
+  return WorkItem{p.full_tiles + piece / p.tail_split, part * per, part * per + per, 0, kb_per_unit, piece};
 }
 
 __device__ __forceinline__ void record_timeout(const GemmParams& p, volatile int* abort, unsigned int where) {
@@ -392,14 +401,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       bool first = true;
       for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
-        const WorkItem it = work_item(w, p);
+        const WorkItem it = work_item(w, p, kb_per_unit);
         int mb, nb;
         tile_coords(it.tile, p, mb, nb);
         const int m0 = mb * Cfg::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
         // this CTA's B rows for MMA width w start at n0 + w * BN
         const int n0 = nb * Cfg::TILE_N + static_cast<int>(rank) * Cfg::SUB_ROWS;
         for (int s = it.s_begin; ok && s < it.s_end; ++s) {
-          for (int i = 0; i < kb_per_unit; ++i) {
+          for (int i = it.i_begin; i < it.i_end; ++i) {
             if ((p.debug_flags & 1u) && !first) {
               ok = false;  // test hook: stop feeding the tensor core after one stage
               break;
@@ -484,7 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0, unit = 0;
       bool ok = true;
       for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
-        const WorkItem it = work_item(w, p);
+        const WorkItem it = work_item(w, p, kb_per_unit);
         for (int s = it.s_begin; ok && s < it.s_end; ++s, ++unit) {
           const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
           if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, abort_flag, budget)) {
@@ -494,7 +503,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after_sync();
           const uint32_t d_tmem = tmem_base + acc * BN;  // ACCS == 1: widths at columns 0 and 256
-          for (int i = 0; i < kb_per_unit; ++i) {
+          for (int i = it.i_begin; i < it.i_end; ++i) {
             if (!mbar_wait(&ctl->full[stage], phase, abort_flag, budget)) {
               record_timeout(p, abort_flag, 0x300u);
               ok = false;
@@ -516,10 +525,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t bw = b_base + w * Cfg::SUB_BYTES;
                 const uint64_t bd = B_MN ? smem_desc_sw128(bw + k * 2048, MN_BOX_BYTES, 1024)
                                          : smem_desc_sw128(bw + k * 32, 16, 1024);
+                const uint32_t accumulate = (i != it.i_begin || k != 0) ? 1u : 0u;
                 if constexpr (PAIR) {
-                  mma_bf16_pair(d_tmem + w * BN, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+                  mma_bf16_pair(d_tmem + w * BN, ad, bd, IDESC, accumulate);
                 } else {
-                  mma_bf16_ss(d_tmem + w * BN, ad, bd, IDESC, (i | k) != 0 ? 1u : 0u);
+                  mma_bf16_ss(d_tmem + w * BN, ad, bd, IDESC, accumulate);
                 }
               }
             }
@@ -569,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t unit = 0;
     bool ok = true;
     for (int w = cluster_id; ok && w < p.num_work; w += num_clusters) {
-      const WorkItem it = work_item(w, p);
+      const WorkItem it = work_item(w, p, kb_per_unit);
       int mb, nb;
       tile_coords(it.tile, p, mb, nb);
       const int row_block = mb * Cfg::CTAS + static_cast<int>(rank);  // this CTA's 128-row block
@@ -647,6 +657,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               p.colsum[static_cast<size_t>(row_block * 4 + q) * p.N + col + lane] = cs;
             }
           } else if constexpr (EPI == EPI_STORE) {
+            if (it.piece >= 0) {
+              // one K piece of a split tile: its fp32 sum goes to the scratch
+              float4* d4 = reinterpret_cast<float4*>(
+                  p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
+                  static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + half * HALF_COLS + c * 32);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              continue;
+            }
             uint32_t op[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) op[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
@@ -667,8 +688,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (s == it.s_end - 1 && it.piece >= 0) {
               // one piece of a split tile: its fp32 sum goes to the scratch
-              float* dst = p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * BN) +
-                           static_cast<size_t>(rank * BM + q * 32 + lane) * BN + half * 128 + c * 32;
+              float* dst = p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
+                           static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + half * 128 + c * 32;
               float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -731,27 +752,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// Finishes the split tiles of a shard-sum GEMM: out[row, col] = bf16(
-// ((piece_0 + piece_1) + ...) + bias[col]), pieces in ascending shard order.
-// One thread per 8 consecutive columns of one row of one split tile.
-template <int TILE_M>
-__global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmParams p) {
-  constexpr int COLS8 = BN / 8;
-  const int tail_tiles = (p.num_work - p.full_tiles) / p.tail_split;
+// Finishes split tiles: out[row, col] = bf16(((piece_0 + piece_1) + ...) +
+// bias[col]) over the pieces of each split tile in order (ascending shards or
+// ascending K).  Split tiles are [first_tile, first_tile + tiles) with
+// `split` pieces each, stored in that order.  One thread per 8 consecutive
+// columns of one row of one split tile.
+template <int TILE_M, int TILE_N>
+__global__ void __launch_bounds__(256) split_reduce_kernel(const GemmParams p, int first_tile, int tiles, int split) {
+  constexpr int COLS8 = TILE_N / 8;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(tail_tiles) * TILE_M * COLS8) return;
+  if (idx >= static_cast<long long>(tiles) * TILE_M * COLS8) return;
   const int t_local = static_cast<int>(idx / (TILE_M * COLS8));
   const int rem = static_cast<int>(idx % (TILE_M * COLS8));
   const int r = rem / COLS8, c8 = (rem % COLS8) * 8;
   int mb, nb;
-  tile_coords(p.full_tiles + t_local, p, mb, nb);
-  const int row = mb * TILE_M + r, col = nb * BN + c8;
+  tile_coords(first_tile + t_local, p, mb, nb);
+  const int row = mb * TILE_M + r, col = nb * TILE_N + c8;
   if (row >= p.M || col >= p.N) return;
   float acc[8];
-  for (int part = 0; part < p.tail_split; ++part) {
+  for (int part = 0; part < split; ++part) {
     const float4* src = reinterpret_cast<const float4*>(
-        p.tail_scratch + static_cast<size_t>(t_local * p.tail_split + part) * (TILE_M * BN) +
-        static_cast<size_t>(r) * BN + c8);
+        p.tail_scratch + static_cast<size_t>(t_local * split + part) * (TILE_M * TILE_N) +
+        static_cast<size_t>(r) * TILE_N + c8);
     const float4 v0 = src[0], v1 = src[1];
     const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll

@@ -120,7 +120,26 @@ size_t tail_pieces_capacity(const Shape& s) {
   return n < TAIL_MAX_PIECES ? n : TAIL_MAX_PIECES;
 }
 size_t tail_offset(const Shape& s) { return partial_offset(s) + partial_bytes(s); }
-size_t workspace_bytes(const Shape& s) { return tail_offset(s) + tail_pieces_capacity(s) * TAIL_PIECE_BYTES; }
+// K pieces of the weight-gradient GEMMs when they have fewer tiles than CTA
+// pairs: at most KSPLIT_MAX_PIECES pieces of 256x512 fp32, and no more than
+// one piece per 8 K slices of every tile.
+constexpr size_t KSPLIT_MAX_PIECES = 128;
+constexpr size_t KSPLIT_PIECE_BYTES = static_cast<size_t>(TileShape::TILE_M) * 512 * sizeof(float);
+size_t ksplit_bytes(const Shape& s) {
+  const size_t kb = 2 * static_cast<size_t>((s.T + BK - 1) / BK);  // two parts (hi, lo)
+  const size_t per_tile = kb / 8;
+  const size_t tiles_dA = static_cast<size_t>((s.h + 255) / 256) * static_cast<size_t>((s.f + 511) / 512);
+  const size_t tiles_dB = static_cast<size_t>((s.f + 255) / 256) * static_cast<size_t>((s.h + 511) / 512);
+  const size_t tiles = tiles_dA > tiles_dB ? tiles_dA : tiles_dB;
+  const size_t pieces = tiles * per_tile < KSPLIT_MAX_PIECES ? tiles * per_tile : KSPLIT_MAX_PIECES;
+  return pieces * KSPLIT_PIECE_BYTES;
+}
+size_t split_scratch_bytes(const Shape& s) {
+  const size_t tail = tail_pieces_capacity(s) * TAIL_PIECE_BYTES;
+  const size_t ks = ksplit_bytes(s);
+  return tail > ks ? tail : ks;
+}
+size_t workspace_bytes(const Shape& s) { return tail_offset(s) + split_scratch_bytes(s); }
 
 // Recomputation keeps Z, H and H_lo in the workspace after the rest:
 // [ ... | Z fp32 | H | H_lo ].
@@ -264,8 +283,8 @@ struct GemmDesc {
   int64_t M, N, K;  // K = shards * (K of one shard); each part spans all of K
   int shards;
   int parts;
-  float* tail_scratch = nullptr;  // shard-sum GEMMs: room for split pieces of the last wave
-  size_t tail_capacity = 0;       // pieces
+  float* tail_scratch = nullptr;  // room for the fp32 pieces of split tiles
+  size_t tail_bytes = 0;
 };
 
 // Tile order.  All resident tiles walk K in near lockstep, so DRAM traffic
@@ -364,13 +383,28 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   // ceil(tail*k/clusters)/k tiles, within the scratch capacity.
   p.full_tiles = p.num_tiles;
   p.tail_split = 1;
-  if (EPI == EPI_SHARD_SUM && p.shards > 1 && g.tail_scratch != nullptr) {
+  p.kb_split = 1;
+  const size_t piece_bytes = static_cast<size_t>(Cfg::TILE_M) * Cfg::TILE_N * sizeof(float);
+  const size_t capacity = g.tail_scratch != nullptr ? g.tail_bytes / piece_bytes : 0;
+  if (EPI == EPI_STORE && p.num_tiles < max_clusters && capacity >= 2) {
+    // fewer tiles than CTA pairs: split every tile's K loop into pieces
+    const int kb_per_unit = p.parts * p.kblocks_per_shard;
+    int k = max_clusters / p.num_tiles;
+    if (k > kb_per_unit / 8) k = kb_per_unit / 8;
+    if (static_cast<size_t>(k) * p.num_tiles > capacity) k = static_cast<int>(capacity / p.num_tiles);
+    if (k >= 2) {
+      p.kb_split = k;
+      p.full_tiles = 0;
+      p.tail_scratch = g.tail_scratch;
+    }
+  }
+  if (EPI == EPI_SHARD_SUM && p.shards > 1 && capacity > 0) {
     const int tail = p.num_tiles % max_clusters;
     if (tail > 0) {
       int best_k = 1;
       double best = 1.0;
       for (int k = 2; k <= p.shards; ++k) {
-        if (p.shards % k != 0 || static_cast<size_t>(tail) * k > g.tail_capacity) continue;
+        if (p.shards % k != 0 || static_cast<size_t>(tail) * k > capacity) continue;
         const double cost = static_cast<double>((tail * k + max_clusters - 1) / max_clusters) / k;
         if (cost < best - 1e-9) {
           best = cost;
@@ -384,7 +418,8 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
       }
     }
   }
-  p.num_work = p.full_tiles + (p.num_tiles - p.full_tiles) * p.tail_split;
+  p.num_work = p.kb_split > 1 ? p.num_tiles * p.kb_split
+                             : p.full_tiles + (p.num_tiles - p.full_tiles) * p.tail_split;
   const int clusters = p.num_work < max_clusters ? p.num_work : max_clusters;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -404,11 +439,15 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
-  if (p.tail_split > 1) {
-    const long long threads = static_cast<long long>(p.num_tiles - p.full_tiles) * Cfg::TILE_M * (BN / 8);
-    tail_reduce_kernel<Cfg::TILE_M><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, L.stream>>>(p);
+  if (p.tail_split > 1 || p.kb_split > 1) {
+    const int first = p.kb_split > 1 ? 0 : p.full_tiles;
+    const int tiles = p.num_tiles - first;
+    const int split = p.kb_split > 1 ? p.kb_split : p.tail_split;
+    const long long threads = static_cast<long long>(tiles) * Cfg::TILE_M * (Cfg::TILE_N / 8);
+    split_reduce_kernel<Cfg::TILE_M, Cfg::TILE_N>
+        <<<static_cast<unsigned>((threads + 255) / 256), 256, 0, L.stream>>>(p, first, tiles, split);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "tail_reduce");
+    if (e != cudaSuccess) return cuda_fail(e, "split_reduce");
     g_launches.fetch_add(1);
   }
   return MLP_OK;
@@ -468,7 +507,20 @@ mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const voi
   p.out1 = static_cast<__nv_bfloat16*>(H_lo);
   p.bias = static_cast<const __nv_bfloat16*>(a);
   GemmDesc g{one(X, false), one(A, true), s.T, s.f, s.h, 1, 1};
-  return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H)");
+  if (kFc1TN == 512) {
+    // 512-column tiles unless their last wave leaves clearly more CTA pairs
+    // idle than 256-column tiles do (full-wave fraction of the two).
+    const int pairs = L.sms / TileShape::CTAS;
+    const int64_t mt = (s.T + TileShape::TILE_M - 1) / TileShape::TILE_M;
+    auto wave_eff = [&](int64_t tn) {
+      const int64_t tiles = mt * ((s.f + tn - 1) / tn);
+      const int64_t waves = (tiles + pairs - 1) / pairs;
+      return static_cast<double>(tiles) / static_cast<double>(waves * pairs);
+    };
+    if (wave_eff(512) + 0.05 >= wave_eff(256))
+      return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H)");
+  }
+  return launch_gemm<false, true, EPI_BIAS_GELU, 256>(g, p, L, "column-parallel forward (Z, H)");
 }
 
 mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const void* B, const void* b, void* Y,
@@ -477,7 +529,7 @@ mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const 
   p.out0 = static_cast<__nv_bfloat16*>(Y);
   p.bias = static_cast<const __nv_bfloat16*>(b);
   GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, s.t, H_lo != nullptr ? 2 : 1,
-             tail_scratch(ws, s), tail_pieces_capacity(s)};
+             tail_scratch(ws, s), split_scratch_bytes(s)};
   return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, L, "row-parallel forward + shard reduce (Y)");
 }
 
@@ -504,7 +556,7 @@ mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* H_lo
   } else {
     GemmParams p = base_params(ws);
     p.out0 = static_cast<__nv_bfloat16*>(dB);
-    GemmDesc g{pair(H, H_lo, true), one(dY, true), s.f, s.h, s.T, 1, 2};
+    GemmDesc g{pair(H, H_lo, true), one(dY, true), s.f, s.h, s.T, 1, 2, tail_scratch(ws, s), split_scratch_bytes(s)};
     st = launch_gemm<true, true, EPI_STORE, kWideTN>(g, p, L, "row-parallel weight gradient (dB)");
   }
   if (st != MLP_OK || db == nullptr) return st;
@@ -516,7 +568,7 @@ mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* dH_lo
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dX);
   GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, s.t, dH_lo != nullptr ? 2 : 1,
-             tail_scratch(ws, s), tail_pieces_capacity(s)};
+             tail_scratch(ws, s), split_scratch_bytes(s)};
   return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, L, "column-parallel backward data + shard reduce (dX)");
 }
 
@@ -525,7 +577,7 @@ mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, 
   if (s.T == 0) return zero_fill(dA, static_cast<size_t>(s.h * s.f * 2), L.stream, "cudaMemsetAsync(dA)");
   GemmParams p = base_params(ws);
   p.out0 = static_cast<__nv_bfloat16*>(dA);
-  GemmDesc g{one(X, true), pair(dH, dH_lo, true), s.h, s.f, s.T, 1, 2};
+  GemmDesc g{one(X, true), pair(dH, dH_lo, true), s.h, s.f, s.T, 1, 2, tail_scratch(ws, s), split_scratch_bytes(s)};
   return launch_gemm<true, true, EPI_STORE, kWideTN>(g, p, L, "column-parallel weight gradient (dA)");
 }
 

@@ -43,6 +43,9 @@ SMALL = [
     (333, 320, 1280, 5),
     (257, 512, 768, 3),
     (130, 128, 512, 8),
+    # few weight-gradient tiles and a long token axis: their K loop is split into pieces
+    (1024, 256, 1024, 2),
+    (2048, 128, 512, 4),
 ]
 
 
@@ -212,3 +215,40 @@ def test_outputs_stay_inside_their_buffers():
         pv = torch.tensor(poison, dtype=buf.dtype)
         assert bool((buf[:pad].cpu() == pv).all()) and bool((buf[pad + n:].cpu() == pv).all()), k
     check_full(out, oracle.full(inputs.make_custom(T, h, f, seed=4)))
+
+
+# ------------------------------------------------------------------ degenerate inputs
+def test_zero_inputs_give_exact_zeros():
+    """X = 0: Z = a, H = g(a) on every row, dA = Xᵀ·dH = 0 exactly.
+    dY = 0: dX, dB, dH, da, db are exactly 0 and dA too."""
+    T, h, f, t = 256, 256, 1024, 4
+    host = inputs.make_custom(T, h, f, seed=41)
+    host["X"].zero_()
+    inp = to_gpu(host)
+    out = run_all(inp, t)
+    assert bool((out["dA"] == 0).all())
+    ref = oracle.full(host)
+    for k in ("Y", "Z", "H", "dX", "da", "dB", "db"):
+        assert_close(k, out[k], ref[k])
+    # every row of Z and H is the same (the bias and its GeLU)
+    assert torch.equal(out["Z"], out["Z"][:1].expand_as(out["Z"]))
+    host2 = inputs.make_custom(T, h, f, seed=42)
+    host2["dY"].zero_()
+    out2 = run_all(to_gpu(host2), t)
+    for k in ("dX", "dA", "da", "dB", "db"):
+        assert bool((out2[k] == 0).all()), k
+    assert_close("Y", out2["Y"], oracle.forward(host2["X"], host2["A"], host2["a"], host2["B"], host2["b"])["Y"])
+
+
+def test_large_preactivations_saturate_gelu():
+    """|Z| up to ~40: GeLU passes positive values through and flushes negative
+    ones to 0, g' goes to 1 and 0; no inf or NaN anywhere."""
+    T, h, f, t = 128, 128, 512, 2
+    host = inputs.make_custom(T, h, f, w_std=0.3, seed=43)
+    host["X"] = (host["X"].float() * 3.0).to(torch.bfloat16)
+    ref = oracle.full(host)
+    assert float(np.abs(ref["Z"]).max()) > 20.0
+    out = run_all(to_gpu(host), t, ALL)
+    for k in out:
+        assert bool(torch.isfinite(out[k].float()).all()), k
+    check_full(out, ref)
