@@ -158,12 +158,22 @@ def oracle_sample_step(inp, rows):
 
 
 def calibrate_oracle_rows(inp, wl, target_s):
-    rows = min(wl.T, 16)
-    t0 = time.perf_counter()
-    oracle_sample_step(inp, rows)
-    dt = time.perf_counter() - t0
-    scaled = int(rows * target_s / max(dt, 1e-3))
-    return max(16, min(wl.T, scaled))
+    """Token rows whose oracle step takes about target_s.  A step costs a
+    fixed part (the fp64 copies of the full weights) plus a part per row, so
+    two timed points fix both."""
+    def timed(rows):
+        t0 = time.perf_counter()
+        oracle_sample_step(inp, rows)
+        return time.perf_counter() - t0
+    r1 = min(wl.T, 16)
+    t1 = timed(r1)
+    r2 = max(r1 + 1, min(wl.T, int(r1 * 0.25 * target_s / max(t1, 1e-3))))
+    if r2 > wl.T:
+        return wl.T
+    t2 = timed(r2)
+    per_row = max((t2 - t1) / (r2 - r1), 1e-9)
+    fixed = max(t1 - per_row * r1, 0.0)
+    return max(16, min(wl.T, int((target_s - fixed) / per_row)))
 
 
 def cpu_baseline(inp, wl, target_s=12.0):
