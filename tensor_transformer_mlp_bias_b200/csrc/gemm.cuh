@@ -20,9 +20,10 @@
 //               16-wide K slice, committing each stage back to the "empty"
 //               barriers of both CTAs and each finished accumulator to their
 //               "tmem full" barriers;
-//   warps 2-9   epilogue: tcgen05.ld the accumulator (one row per thread,
-//               32 columns per load), apply the fused math, store to global
-//               memory, release the accumulator.
+//   warps 2-    epilogue (8 or 16 warps, see TileCfg):
+//               tcgen05.ld the accumulator (one row per thread, 32 columns
+//               per load), apply the fused math, store to global memory,
+//               release the accumulator.
 // The two accumulators let the epilogue of one unit overlap the mainloop of
 // the next.
 //
@@ -65,8 +66,6 @@ constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
 constexpr int MN_BOX_BYTES = 64 * BK * 2;   // one 64x64 bf16 box, 8 KB
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int CTL_BYTES = 1024;
 
@@ -88,8 +87,12 @@ __host__ __device__ constexpr int epi_warp_bytes(int epi) {
 // all 512 TMEM columns).  The wide tile reads 25% fewer operand bytes per
 // FLOP from L2, which is what bounds these GEMMs without TMA multicast.
 // STAGES is the shared-memory pipeline depth (BK-wide K slices in flight):
-// as many as fit beside the epilogue staging.
-template <bool PAIR, int TN, int EPI>
+// as many as fit beside the epilogue staging.  EW is the number of epilogue
+// warps, 8 or 16: four lane quadrants times 2 or 4 column slices.  Sixteen
+// keep twice as many chunks in flight per scheduler, which pays where the
+// epilogue (waiting on TMEM and global loads) outlasts a short mainloop, at
+// the cost of staging space, i.e. pipeline stages.
+template <bool PAIR, int TN, int EPI, int EW = 8>
 struct TileCfg {
   static_assert(TN == 256 || (TN == 512 && PAIR), "wide tiles need a CTA pair");
   static constexpr int CTAS = PAIR ? 2 : 1;
@@ -102,7 +105,11 @@ struct TileCfg {
   static constexpr int SUB_BYTES = SUB_ROWS * BK * 2;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // one CTA's share of a stage
-  static constexpr int EPI_BYTES = NUM_EPI_WARPS * epi_warp_bytes(EPI);
+  static constexpr int EPI_WARPS = EW;
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;          // producer, MMA issuer, epilogue
+  static constexpr int SLICE_COLS = TN / (EPI_WARPS / 4);      // columns per epilogue warp (4 lane quadrants)
+  static_assert(EPI_WARPS % 4 == 0 && SLICE_COLS % 32 == 0, "epilogue warps must tile the accumulator");
+  static constexpr int EPI_BYTES = EPI_WARPS * epi_warp_bytes(EPI);
   static constexpr int SMEM_LIMIT = 227 * 1024;
   static constexpr int FIXED = EPI_BYTES + CTL_BYTES + 1024;   // + alignment slack
   static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED) / STAGE_BYTES;
@@ -253,13 +260,17 @@ __device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t& hi, u
   lo = pack_bf16x2(v0 - h.x, v1 - h.y);
 }
 
-// 32 consecutive bf16 values -> fp32 (vectorised 16-byte loads).
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&dst)[32]) {
+// 32 consecutive bf16 values: raw 16-byte loads, then widening to fp32.
+__device__ __forceinline__ void load_bf16x32_raw(const __nv_bfloat16* src, uint4 (&w)[4]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
+  for (int v = 0; v < 4; ++v) w[v] = __ldg(s + v);
+}
+
+__device__ __forceinline__ void widen_bf16x32(const uint4 (&w)[4], float (&dst)[32]) {
+#pragma unroll
   for (int v = 0; v < 4; ++v) {
-    const uint4 w = __ldg(s + v);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t u[4] = {w[v].x, w[v].y, w[v].z, w[v].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = unpack_bf16x2(u[e]);
@@ -267,6 +278,12 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&d
       dst[v * 8 + 2 * e + 1] = f.y;
     }
   }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&dst)[32]) {
+  uint4 w[4];
+  load_bf16x32_raw(src, w);
+  widen_bf16x32(w, dst);
 }
 
 __device__ __forceinline__ void load_f32x32(const float* src, float (&dst)[32]) {
@@ -322,10 +339,10 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- kernel
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW>
+__global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
-  using Cfg = TileCfg<PAIR, TN, EPI>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
   static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
   constexpr int ACCS = Cfg::ACCS;
   constexpr int STAGES = Cfg::STAGES;
@@ -353,7 +370,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
     for (int a = 0; a < ACCS; ++a) {
       mbar_init(&ctl->tfull[a], 1);
-      mbar_init(&ctl->tempty[a], NUM_EPI_WARPS * Cfg::CTAS);  // every epilogue warp of the pair
+      mbar_init(&ctl->tempty[a], Cfg::EPI_WARPS * Cfg::CTAS);  // every epilogue warp of the pair
     }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort = 0;
@@ -563,8 +580,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int q = warp & 3;     // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;   // column half of the tile (TN/2 columns)
-    constexpr int HALF_COLS = Cfg::TILE_N / 2;
+    const int slice = ew >> 2;  // column slice of the tile (SLICE_COLS columns)
+    constexpr int SLICE_COLS = Cfg::SLICE_COLS;
     // the MMA issuer's "accumulator drained" barriers (in the leader CTA)
     // this warp's staging tiles: [fp32 (EPI_BIAS_GELU)] [bf16 out0] [bf16 out1]
     const uint32_t stage_base = smem_u32(sEpi + ew * epi_warp_bytes(EPI));
@@ -586,9 +603,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row0 = row_block * BM + q * 32;  // this warp's first row
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
-      float sum[EPI == EPI_SHARD_SUM ? 128 : 1];
+      float sum[EPI == EPI_SHARD_SUM ? SLICE_COLS : 1];
       for (int s = it.s_begin; s < it.s_end; ++s, ++unit) {
         const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
+        // bias+GeLU on wide tiles (single accumulator, epilogue not hidden):
+        // the first chunk's bias is fetched while the mainloop runs, each
+        // later chunk's during the chunk before it
+        constexpr bool BIAS_AHEAD = EPI == EPI_BIAS_GELU && TN == 512;
+        uint4 bias_raw[BIAS_AHEAD ? 4 : 1];
+        if constexpr (BIAS_AHEAD) {
+          const int col0 = nb * Cfg::TILE_N + slice * SLICE_COLS;
+          if (col0 < p.N) load_bf16x32_raw(p.bias + col0, bias_raw);
+        }
         if (!mbar_wait(&ctl->tfull[acc], acc_phase, abort_flag, budget)) {
           record_timeout(p, abort_flag, 0x400u);
           ok = false;
@@ -596,10 +622,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after_sync();
         const uint32_t t_addr =
-            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * HALF_COLS;
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + slice * SLICE_COLS;
 #pragma unroll
-        for (int c = 0; c < HALF_COLS / 32; ++c) {
-          const int col = nb * Cfg::TILE_N + half * HALF_COLS + c * 32;
+        for (int c = 0; c < SLICE_COLS / 32; ++c) {
+          const int col = nb * Cfg::TILE_N + slice * SLICE_COLS + c * 32;
           if (col >= p.N) continue;  // warp-uniform: ragged last column block
           uint32_t r[32];
           tmem_load_32cols(t_addr + c * 32, r);
@@ -610,7 +636,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if constexpr (EPI == EPI_BIAS_GELU) {
             // Z = X·A + a (fp32, saved), H = g(Z) saved as (hi, lo)
             float bias[32];
-            load_bf16x32(p.bias + col, bias);
+            if constexpr (BIAS_AHEAD) {
+              widen_bf16x32(bias_raw, bias);
+              if (c + 1 < SLICE_COLS / 32 && col + 32 < p.N) load_bf16x32_raw(p.bias + col + 32, bias_raw);
+            } else {
+              load_bf16x32(p.bias + col, bias);
+            }
             float z[32];
             uint32_t hp[16], lp[16];
 #pragma unroll
@@ -661,7 +692,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               // one K piece of a split tile: its fp32 sum goes to the scratch
               float4* d4 = reinterpret_cast<float4*>(
                   p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
-                  static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + half * HALF_COLS + c * 32);
+                  static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS + c * 32);
 #pragma unroll
               for (int j = 0; j < 8; ++j)
                 d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
@@ -689,7 +720,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (s == it.s_end - 1 && it.piece >= 0) {
               // one piece of a split tile: its fp32 sum goes to the scratch
               float* dst = p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
-                           static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + half * 128 + c * 32;
+                           static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS + c * 32;
               float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
               for (int j = 0; j < 8; ++j)

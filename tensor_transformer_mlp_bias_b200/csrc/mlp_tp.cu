@@ -91,6 +91,10 @@ constexpr int kWideTN = kPair ? MLPTP_WIDE_TN : 256;
 #endif
 constexpr int kFc1TN = kPair ? MLPTP_FC1_TN : 256;    // bias+GeLU GEMM
 constexpr int kFc2BdTN = kPair ? MLPTP_FC2BD_TN : 256;  // GeLU-derivative GEMM
+#ifndef MLPTP_FC2BD_MANY_WARPS_MAX_K
+#define MLPTP_FC2BD_MANY_WARPS_MAX_K 3072
+#endif
+constexpr int64_t kFc2BdManyWarpsMaxK = MLPTP_FC2BD_MANY_WARPS_MAX_K;
 using TileShape = TileCfg<kPair, 256, EPI_STORE>;
 // 128-row blocks that a GEMM over R rows covers (whole tiles).
 size_t gemm_row_blocks(int64_t R) {
@@ -302,13 +306,13 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
 
 // One opt-in per kernel instantiation and device (the static state is per
 // template instance).
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW>
 mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
-  using Cfg = TileCfg<PAIR, TN, EPI>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
   static std::mutex mu;
   static uint64_t done_mask = 0;
   static int clusters[64] = {};
-  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN>;
+  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW>;
   std::lock_guard<std::mutex> lk(mu);
   if (!(done_mask & (1ull << dev))) {
     cudaError_t e =
@@ -323,7 +327,7 @@ mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(static_cast<unsigned>(2 * n));
-      cfg.blockDim = dim3(NUM_THREADS);
+      cfg.blockDim = dim3(Cfg::THREADS);
       cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
@@ -344,9 +348,9 @@ struct Launch {
   cudaStream_t stream;
 };
 
-template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair>
+template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
-  using Cfg = TileCfg<PAIR, TN, EPI>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
   if (g.M == 0 || g.N == 0) return MLP_OK;
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -374,26 +378,42 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.debug_flags = g_debug_flags.load();
 
   int max_clusters = 0;
-  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN>(L.dev, L.sms, &max_clusters);
+  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN, EW>(L.dev, L.sms, &max_clusters);
   if (st != MLP_OK) return st;
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
-  // Work list.  A shard-sum GEMM whose last wave is partial splits each tile
-  // of that wave into k pieces of shards/k consecutive shards, k a divisor of
-  // the shard count chosen to minimise the time of that wave,
-  // ceil(tail*k/clusters)/k tiles, within the scratch capacity.
+  // Work list.  Split pieces trade idle CTA pairs for extra traffic: a piece
+  // stores its fp32 partial (TILE_M x TILE_N x 4 bytes) to scratch and a
+  // reduce pass reads it back.  Costs are in K-slice units (one BK slice of a
+  // tile's MMA); a whole tile runs U slices, a piece U/k plus
+  // kPieceOverheadSlices for its store and read-back (all pairs storing
+  // 256 KB at ~6 TB/s take ~3 us, about 9 slices at 1.5 GHz; measured on
+  // B200: 4-way pieces of 16 slices made a 64-slice shard-sum GEMM slower).
+  //  - EPI_STORE with fewer tiles than CTA pairs: every tile's K loop is cut
+  //    into k pieces of consecutive K slices.
+  //  - EPI_SHARD_SUM whose last wave is partial: each tile of that wave is
+  //    cut into k pieces of shards/k consecutive shards (k divides t).
+  // k minimises rounds(items) x (U/k + overhead) within the scratch capacity.
+  constexpr double kPieceOverheadSlices = 12.0;
   p.full_tiles = p.num_tiles;
   p.tail_split = 1;
   p.kb_split = 1;
   const size_t piece_bytes = static_cast<size_t>(Cfg::TILE_M) * Cfg::TILE_N * sizeof(float);
   const size_t capacity = g.tail_scratch != nullptr ? g.tail_bytes / piece_bytes : 0;
+  const int kb_per_unit = p.parts * p.kblocks_per_shard;  // slices per shard
+  auto rounds = [&](long long items) { return static_cast<double>((items + max_clusters - 1) / max_clusters); };
   if (EPI == EPI_STORE && p.num_tiles < max_clusters && capacity >= 2) {
-    // fewer tiles than CTA pairs: split every tile's K loop into pieces
-    const int kb_per_unit = p.parts * p.kblocks_per_shard;
-    int k = max_clusters / p.num_tiles;
-    if (k > kb_per_unit / 8) k = kb_per_unit / 8;
-    if (static_cast<size_t>(k) * p.num_tiles > capacity) k = static_cast<int>(capacity / p.num_tiles);
-    if (k >= 2) {
-      p.kb_split = k;
+    const double U = kb_per_unit;
+    int best_k = 1;
+    double best = U;
+    for (int k = 2; k <= kb_per_unit / 8 && static_cast<size_t>(k) * p.num_tiles <= capacity; ++k) {
+      const double cost = rounds(static_cast<long long>(p.num_tiles) * k) * (U / k + kPieceOverheadSlices);
+      if (cost < best - 1e-9) {
+        best = cost;
+        best_k = k;
+      }
+    }
+    if (best_k > 1) {
+      p.kb_split = best_k;
       p.full_tiles = 0;
       p.tail_scratch = g.tail_scratch;
     }
@@ -401,11 +421,12 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   if (EPI == EPI_SHARD_SUM && p.shards > 1 && capacity > 0) {
     const int tail = p.num_tiles % max_clusters;
     if (tail > 0) {
+      const double U = static_cast<double>(p.shards) * kb_per_unit;
       int best_k = 1;
-      double best = 1.0;
+      double best = U;
       for (int k = 2; k <= p.shards; ++k) {
         if (p.shards % k != 0 || static_cast<size_t>(tail) * k > capacity) continue;
-        const double cost = static_cast<double>((tail * k + max_clusters - 1) / max_clusters) / k;
+        const double cost = rounds(static_cast<long long>(tail) * k) * (U / k + kPieceOverheadSlices);
         if (cost < best - 1e-9) {
           best = cost;
           best_k = k;
@@ -430,12 +451,12 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * Cfg::CTAS));
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(Cfg::THREADS);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = L.stream;
   cfg.attrs = attr;
   cfg.numAttrs = PAIR ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN>, maps, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW>, maps, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
@@ -543,7 +564,13 @@ mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, co
   p.aux = static_cast<const float*>(Z);
   p.colsum = da != nullptr ? partials(ws, s) : nullptr;
   GemmDesc g{one(dY, false), one(B, false), s.T, s.f, s.h, 1, 1};
-  mlp_status_t st = launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN>(g, p, L, "row-parallel backward data (dH, da)");
+  // 16 epilogue warps when K = h is short enough for the epilogue (loads of
+  // Z, g'(Z), the dH pair, column sums) to outlast the mainloop of a tile:
+  // measured on B200, 24% faster at h = 1024, 1.4% slower at h = 4096.
+  mlp_status_t st =
+      s.h <= kFc2BdManyWarpsMaxK
+          ? launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 16>(g, p, L, "row-parallel backward data (dH, da)")
+          : launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 8>(g, p, L, "row-parallel backward data (dH, da)");
   if (st != MLP_OK || da == nullptr) return st;
   return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream);
 }
