@@ -237,7 +237,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--split", type=int, default=0,
                     help="split flags: 1 = Y from the (H, H_lo) pair, 2 = dX from the (dH, dH_lo) pair")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-t", action="store_true", help="time only the headline shard count")
     ap.add_argument("--clock-interval-ms", type=int, default=100,

@@ -39,7 +39,10 @@
 // is kept as a bf16 pair v = hi + lo (hi = bf16(v), lo = bf16(v - hi), about
 // 16 significant bits).  A product that must see that precision runs its K
 // loop twice ("parts"): once over (hi, other operand) and once over
-// (lo, other operand), accumulating into the same TMEM accumulator.
+// (lo, other operand), accumulating into the same TMEM accumulator.  With
+// DUAL, the split operand is A and both halves ride in the same stage: one
+// pass over K loads A_hi, A_lo and B once and issues both products per K
+// slice, so B crosses from L2 once instead of twice.
 //
 // Operand layouts.  A K-major operand is stored [rows, K] with K contiguous
 // and arrives as one TMA box of 64 (K) x rows.  An MN-major operand is
@@ -92,7 +95,7 @@ __host__ __device__ constexpr int epi_warp_bytes(int epi) {
 // keep twice as many chunks in flight per scheduler, which pays where the
 // epilogue (waiting on TMEM and global loads) outlasts a short mainloop, at
 // the cost of staging space, i.e. pipeline stages.
-template <bool PAIR, int TN, int EPI, int EW = 8>
+template <bool PAIR, int TN, int EPI, int EW = 8, bool DUAL = false>
 struct TileCfg {
   static_assert(TN == 256 || (TN == 512 && PAIR), "wide tiles need a CTA pair");
   static constexpr int CTAS = PAIR ? 2 : 1;
@@ -104,7 +107,8 @@ struct TileCfg {
   static constexpr int B_ROWS = SUB_ROWS * WIDTHS;             // B operand rows held by one CTA
   static constexpr int SUB_BYTES = SUB_ROWS * BK * 2;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
-  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // one CTA's share of a stage
+  static constexpr int A_BYTES = A_STAGE_BYTES * (DUAL ? 2 : 1);      // A (and A_lo with DUAL)
+  static constexpr int STAGE_BYTES = A_BYTES + B_STAGE_BYTES;          // one CTA's share of a stage
   static constexpr int EPI_WARPS = EW;
   static constexpr int THREADS = 64 + EPI_WARPS * 32;          // producer, MMA issuer, epilogue
   static constexpr int SLICE_COLS = TN / (EPI_WARPS / 4);      // columns per epilogue warp (4 lane quadrants)
@@ -339,10 +343,11 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- kernel
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW>
-__global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL>
+__global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
-  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
+  static_assert(!DUAL || PAIR, "both halves of A in one stage: pair mode");
   static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
   constexpr int ACCS = Cfg::ACCS;
   constexpr int STAGES = Cfg::STAGES;
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
   uint8_t* sEpi = smem + STAGES * Cfg::STAGE_BYTES;  // 1024-aligned: STAGE_BYTES is a multiple of 1024
   GemmCtl* ctl = reinterpret_cast<GemmCtl*>(sEpi + Cfg::EPI_BYTES);
 
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
             const int k0 = (s * p.kblocks_per_shard + (i - part * p.kblocks_per_shard)) * BK;
             const CUtensorMap* ma = &maps.a[part];
             const CUtensorMap* mbp = &maps.b[part];
-            const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
+            const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
             const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
             if constexpr (PAIR) {
               const uint32_t fb = map_shared_to_cta(smem_u32(&ctl->full[stage]), 0u);
@@ -452,8 +457,13 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
               if (A_MN) {
                 tma_load_2d_pair(a_dst, ma, fb, m0, k0);
                 tma_load_2d_pair(a_dst + MN_BOX_BYTES, ma, fb, m0 + 64, k0);
+                if constexpr (DUAL) {  // the low half of A, same rows and K slice
+                  tma_load_2d_pair(a_dst + A_STAGE_BYTES, &maps.a[1], fb, m0, k0);
+                  tma_load_2d_pair(a_dst + A_STAGE_BYTES + MN_BOX_BYTES, &maps.a[1], fb, m0 + 64, k0);
+                }
               } else {
                 tma_load_2d_pair(a_dst, ma, fb, k0, m0);
+                if constexpr (DUAL) tma_load_2d_pair(a_dst + A_STAGE_BYTES, &maps.a[1], fb, k0, m0);
               }
 #pragma unroll
               for (int w = 0; w < Cfg::WIDTHS; ++w) {
@@ -527,7 +537,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
               break;
             }
             tc_fence_after_sync();
-            const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
+            const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
             const uint32_t b_base = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
@@ -545,6 +555,12 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW>::THREADS, 1)
                 const uint32_t accumulate = (i != it.i_begin || k != 0) ? 1u : 0u;
                 if constexpr (PAIR) {
                   mma_bf16_pair(d_tmem + w * BN, ad, bd, IDESC, accumulate);
+                  if constexpr (DUAL) {  // the low half of A into the same accumulator
+                    const uint32_t alo = a_base + A_STAGE_BYTES;
+                    const uint64_t ad_lo = A_MN ? smem_desc_sw128(alo + k * 2048, MN_BOX_BYTES, 1024)
+                                                : smem_desc_sw128(alo + k * 32, 16, 1024);
+                    mma_bf16_pair(d_tmem + w * BN, ad_lo, bd, IDESC, 1u);
+                  }
                 } else {
                   mma_bf16_ss(d_tmem + w * BN, ad, bd, IDESC, accumulate);
                 }

@@ -95,6 +95,12 @@ constexpr int kFc2BdTN = kPair ? MLPTP_FC2BD_TN : 256;  // GeLU-derivative GEMM
 #define MLPTP_FC2BD_MANY_WARPS_MAX_K 3072
 #endif
 constexpr int64_t kFc2BdManyWarpsMaxK = MLPTP_FC2BD_MANY_WARPS_MAX_K;
+// GEMMs whose A operand is a (hi, lo) pair carry both halves in one stage
+// (one pass over K, B read once).
+#ifndef MLPTP_DUAL_A
+#define MLPTP_DUAL_A 1
+#endif
+constexpr bool kDualA = kPair && MLPTP_DUAL_A != 0;
 using TileShape = TileCfg<kPair, 256, EPI_STORE>;
 // 128-row blocks that a GEMM over R rows covers (whole tiles).
 size_t gemm_row_blocks(int64_t R) {
@@ -306,13 +312,13 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
 
 // One opt-in per kernel instantiation and device (the static state is per
 // template instance).
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL>
 mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
-  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   static std::mutex mu;
   static uint64_t done_mask = 0;
   static int clusters[64] = {};
-  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW>;
+  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>;
   std::lock_guard<std::mutex> lk(mu);
   if (!(done_mask & (1ull << dev))) {
     cudaError_t e =
@@ -348,9 +354,9 @@ struct Launch {
   cudaStream_t stream;
 };
 
-template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8>
+template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8, bool DUAL = false>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
-  using Cfg = TileCfg<PAIR, TN, EPI, EW>;
+  using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   if (g.M == 0 || g.N == 0) return MLP_OK;
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -369,7 +375,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.M = static_cast<int>(g.M);
   p.N = static_cast<int>(g.N);
   p.shards = g.shards;
-  p.parts = g.parts;
+  p.parts = DUAL ? 1 : g.parts;  // DUAL: both halves of A in each stage, one pass over K
   p.kblocks_per_shard = static_cast<int>((g.K / g.shards + BK - 1) / BK);
   p.m_blocks = static_cast<int>((g.M + Cfg::TILE_M - 1) / Cfg::TILE_M);
   p.n_blocks = static_cast<int>((g.N + Cfg::TILE_N - 1) / Cfg::TILE_N);
@@ -378,7 +384,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.debug_flags = g_debug_flags.load();
 
   int max_clusters = 0;
-  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN, EW>(L.dev, L.sms, &max_clusters);
+  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>(L.dev, L.sms, &max_clusters);
   if (st != MLP_OK) return st;
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
   // Work list.  Split pieces trade idle CTA pairs for extra traffic: a piece
@@ -456,7 +462,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   cfg.stream = L.stream;
   cfg.attrs = attr;
   cfg.numAttrs = PAIR ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW>, maps, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>, maps, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
@@ -551,6 +557,8 @@ mlp_status_t fc2_forward(const Shape& s, const void* H, const void* H_lo, const 
   p.bias = static_cast<const __nv_bfloat16*>(b);
   GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, s.t, H_lo != nullptr ? 2 : 1,
              tail_scratch(ws, s), split_scratch_bytes(s)};
+  if (H_lo != nullptr)
+    return launch_gemm<false, true, EPI_SHARD_SUM, 256, kPair, 8, kDualA>(g, p, L, "row-parallel forward + shard reduce (Y)");
   return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, L, "row-parallel forward + shard reduce (Y)");
 }
 
@@ -584,7 +592,7 @@ mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* H_lo
     GemmParams p = base_params(ws);
     p.out0 = static_cast<__nv_bfloat16*>(dB);
     GemmDesc g{pair(H, H_lo, true), one(dY, true), s.f, s.h, s.T, 1, 2, tail_scratch(ws, s), split_scratch_bytes(s)};
-    st = launch_gemm<true, true, EPI_STORE, kWideTN>(g, p, L, "row-parallel weight gradient (dB)");
+    st = launch_gemm<true, true, EPI_STORE, kWideTN, kPair, 8, kDualA>(g, p, L, "row-parallel weight gradient (dB)");
   }
   if (st != MLP_OK || db == nullptr) return st;
   return launch_colsum(dY, s.T, s.h, db, partials(ws, s), L.stream);
@@ -596,6 +604,9 @@ mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* dH_lo
   p.out0 = static_cast<__nv_bfloat16*>(dX);
   GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, s.t, dH_lo != nullptr ? 2 : 1,
              tail_scratch(ws, s), split_scratch_bytes(s)};
+  if (dH_lo != nullptr)
+    return launch_gemm<false, false, EPI_SHARD_SUM, 256, kPair, 8, kDualA>(
+        g, p, L, "column-parallel backward data + shard reduce (dX)");
   return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, L, "column-parallel backward data + shard reduce (dX)");
 }
 
