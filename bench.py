@@ -240,6 +240,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-t", action="store_true", help="time only the headline shard count")
+    ap.add_argument("--no-recompute", action="store_true", help="skip the activation-recomputation leg")
     ap.add_argument("--clock-interval-ms", type=int, default=100,
                     help="nvidia-smi sampling period during the timed region")
     args = ap.parse_args()
@@ -357,6 +358,40 @@ def main():
         del ws_o
     per_t[str(t)] = {"value": value, "ms_per_step": ms_per_step, "steps": args.steps}
 
+    # ------------------------------------------------ activation recomputation
+    # mlp_tp_forward_recompute + mlp_tp_backward_recompute on the same inputs:
+    # nothing of size T·f outlives the forward, and the backward reruns the
+    # column-parallel GEMM.  Throughput counts the block's algorithmic FLOPs
+    # only (the rerun GEMM is overhead, not work).
+    recompute = None
+    if not args.no_recompute:
+        ws_r = binding.make_recompute_workspace(T, h, f, t)
+
+        def step_r():
+            binding.mlp_tp_forward_recompute(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, split,
+                                             Y, ws_r, sh)
+            binding.mlp_tp_backward_recompute(dev["dY"], dev["X"], dev["A"], dev["a"], dev["B"], T, h, f, t, split,
+                                              dX, dA, da, dB, db, ws_r, sh)
+
+        for _ in range(3):
+            step_r()
+        n_r = max(10, args.steps // 4)
+        s_r, e_r = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        s_r.record(stream)
+        for _ in range(n_r):
+            step_r()
+        e_r.record(stream)
+        torch.cuda.synchronize()
+        binding.mlp_tp_check(ws_r, sh)
+        ms_r, fl_r = reduce_max_sum(s_r.elapsed_time(e_r), float(wl.flops) * n_r)
+        recompute = {"value": fl_r / (ms_r * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_r / n_r, "steps": n_r,
+                     "extra_gemm_flops_per_step": 2.0 * T * h * f,
+                     "saved_activation_bytes_avoided": 8 * T * f,
+                     "api": "mlp_tp_forward_recompute + mlp_tp_backward_recompute, inputs resident on the device"}
+        del ws_r
+
     # ------------------------------------------------ end-to-end through the public API
     # Each step copies its inputs from pinned host memory, runs mlp_tp_forward
     # and mlp_tp_backward, and copies its outputs back to pinned host memory.
@@ -471,6 +506,8 @@ def main():
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if recompute is not None:
+        line["recompute"] = recompute
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(host, wl)
     print(json.dumps(line), flush=True)

@@ -321,6 +321,38 @@ __device__ __forceinline__ void stage_f32x32(uint32_t tile, int r, const float (
                  __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
 }
 
+// This lane's row of the 32x32 fp32 block at (row0, col) of a row-major
+// [M, N] matrix, read coalesced: eight lanes cover one 128-byte row segment
+// (4 rows per load instruction, 8 instructions), the block is transposed
+// through `tile` (4 KB of the warp's staging, free on entry: 128-byte rows,
+// chunk j of row r at chunk j ^ (r & 7), so both the writes and the per-row
+// reads hit every bank), and each lane reads back its own row.  Reading the
+// rows one per lane instead touches 32 cache lines per instruction.  Rows
+// at or past M read as 0.  `tile` is free again on return.
+__device__ __forceinline__ void load_rows_f32x32_coalesced(const float* src, int M, int N, int row0, int col,
+                                                           uint32_t tile, int lane, float (&dst)[32]) {
+  const int rr = lane >> 3, cc = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = i * 4 + rr;
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (row0 + r < M)
+      v = __ldg(reinterpret_cast<const float4*>(src + static_cast<size_t>(row0 + r) * static_cast<size_t>(N) + col) + cc);
+    st_shared_v4(tile + r * 128 + ((cc ^ (r & 7)) << 4), __float_as_uint(v.x), __float_as_uint(v.y),
+                 __float_as_uint(v.z), __float_as_uint(v.w));
+  }
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 v = ld_shared_v4f(tile + lane * 128 + ((j ^ (lane & 7)) << 4));
+    dst[4 * j] = v.x;
+    dst[4 * j + 1] = v.y;
+    dst[4 * j + 2] = v.z;
+    dst[4 * j + 3] = v.w;
+  }
+  __syncwarp();
+}
+
 // Column sums over the warp's 32 rows: lane r holds row r's 32 values; on
 // return lane j holds the sum over rows of column j.  Recursive halving:
 // at each step a lane keeps the half of its columns selected by one bit of
@@ -678,12 +710,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
           } else if constexpr (EPI == EPI_GELU_GRAD) {
             // dH = (dY·Bᵀ) ⊙ g'(Z), saved as (hi, lo); fp32 column sums for da
             float z[32];
-            if (row_ok) {
-              load_f32x32(p.aux + static_cast<size_t>(row) * static_cast<size_t>(p.N) + col, z);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) z[j] = 0.0f;
-            }
+            load_rows_f32x32_coalesced(p.aux, p.M, p.N, row0, col, stage_base, lane, z);
             float dh[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) dh[j] = row_ok ? __uint_as_float(r[j]) * gelu_grad_f(z[j]) : 0.0f;
