@@ -1,0 +1,105 @@
+"""Cross-GPU orchestration of the block (tensor_transformer_mlp_bias_b200.tp)
+as two gloo ranks on the CPU.
+
+Each rank holds one shard (its column block of A and a, its row block of B)
+and runs the stage calls through the fp64 stand-in in tests/tp_cpu_ops.py;
+the collectives are torch.distributed's.  Every rank checks its results
+against the oracle's unsharded block: Y and dX (all-reduced, or its token
+rows in the sequence-parallel form), its shard of dA, da and dB, and db.
+This pins the host logic: which rank adds b, which outputs are reduced,
+gathered or scattered, and the shard and token bounds.  The GEMMs are
+checked on the GPU elsewhere; runs on several GPUs are not possible on a
+one-GPU machine.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from tensor_transformer_mlp_bias_b200 import tp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, shape, sp, split, results):
+    import torch.distributed as dist
+    from oracle import mlp_oracle as oracle
+    from tensor_transformer_mlp_bias_b200 import inputs
+    from tests import tp_cpu_ops
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        T, h, f = shape
+        inp = inputs.make_custom(T, h, f, seed=11)
+        ref = oracle.full(inp)
+        d = {k: v.to(torch.float64) for k, v in inp.items()}
+        A_i, a_i, B_i = tp.shard_parameters(d["A"], d["a"], d["B"], rank, world)
+        lo, hi = tp.shard_bounds(f, rank, world)
+        rows = tp.token_rows(T, rank, world) if sp else slice(0, T)
+        X = d["X"][rows] if sp else d["X"]
+        dY = d["dY"][rows] if sp else d["dY"]
+        Y, saved = tp.forward(X, A_i, a_i, B_i, d["b"], sequence_parallel=sp, split=split, ops=tp_cpu_ops)
+        g = tp.backward(dY, saved, A_i, B_i, sequence_parallel=sp, split=split, ops=tp_cpu_ops)
+        err = {
+            "Y": np.abs(Y.numpy() - ref["Y"][rows]).max(),
+            "dX": np.abs(g["dX"].numpy() - ref["dX"][rows]).max(),
+            "dA": np.abs(g["dA"].numpy() - ref["dA"][:, lo:hi]).max(),
+            "da": np.abs(g["da"].numpy() - ref["da"][lo:hi]).max(),
+            "dB": np.abs(g["dB"].numpy() - ref["dB"][lo:hi, :]).max(),
+            "db": np.abs(g["db"].numpy() - ref["db"]).max(),
+        }
+        scale = {k: 1.0 + float(np.abs(ref[k]).max()) for k in err}
+        results[rank] = {k: float(v) / scale[k] for k, v in err.items()}
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, shape, sp, split):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    results = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, shape, sp, split, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    return dict(results)
+
+
+@pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
+@pytest.mark.parametrize("split", [0, 3], ids=["split_none", "split_all"])
+def test_two_ranks_match_the_unsharded_block(sp, split):
+    res = _run(2, (64, 128, 256), sp, split)
+    assert set(res) == {0, 1}
+    for rank, errs in res.items():
+        for k, e in errs.items():
+            assert e < 1e-12, (rank, k, e)
+
+
+def test_shard_and_token_bounds():
+    assert tp.shard_bounds(1024, 0, 4) == (0, 256)
+    assert tp.shard_bounds(1024, 3, 4) == (768, 1024)
+    assert tp.token_rows(64, 1, 2) == slice(32, 64)
+    with pytest.raises(ValueError):
+        tp.shard_bounds(1000, 0, 3)
+    with pytest.raises(ValueError):
+        tp.token_rows(63, 0, 2)
+    A = torch.arange(4 * 8, dtype=torch.float64).view(4, 8)
+    a = torch.arange(8, dtype=torch.float64)
+    B = torch.arange(8 * 4, dtype=torch.float64).view(8, 4)
+    A1, a1, B1 = tp.shard_parameters(A, a, B, 1, 2)
+    assert torch.equal(A1, A[:, 4:]) and torch.equal(a1, a[4:]) and torch.equal(B1, B[4:, :])
+    assert A1.is_contiguous() and B1.is_contiguous()

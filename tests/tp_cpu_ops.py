@@ -1,0 +1,66 @@
+"""Test stand-in for the C-ABI stage calls on the CPU, in fp64, for the
+multi-process tests of the cross-GPU orchestration in
+tensor_transformer_mlp_bias_b200.tp.  Same call signatures as the binding.
+
+It computes each stage from the oracle's definitions (GeLU and its derivative
+from oracle/mlp_oracle.py, plain matrix products), writing into the output
+tensors it is given.  It holds everything in fp64, so the low halves of the
+activation pairs are 0.  This is test infrastructure: the library never
+falls back to it.
+"""
+import numpy as np
+import torch
+
+from oracle import mlp_oracle as oracle
+
+DTYPE = torch.float64
+Z_DTYPE = torch.float64
+
+
+def _np(x):
+    return x.detach().numpy()
+
+
+def make_workspace(T, h, f, t, device=None):
+    return None
+
+
+def mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, H_lo, ws, stream=None):
+    z = _np(X) @ _np(A) + _np(a)
+    Z.copy_(torch.from_numpy(z))
+    H.copy_(torch.from_numpy(oracle.gelu(z)))
+    H_lo.zero_()
+
+
+def mlp_tp_fc2_forward(H, H_lo, B, b, T, h, f, t, Y, ws, stream=None):
+    hh = _np(H) + (_np(H_lo) if H_lo is not None else 0.0)
+    y = hh @ _np(B)
+    if b is not None:
+        y = y + _np(b)
+    Y.copy_(torch.from_numpy(y))
+
+
+def mlp_tp_fc2_backward_data(dY, B, Z, T, h, f, t, dH, dH_lo, da, ws, stream=None):
+    dh = (_np(dY) @ _np(B).T) * oracle.gelu_grad(_np(Z))
+    dH.copy_(torch.from_numpy(dh))
+    if dH_lo is not None:
+        dH_lo.zero_()
+    if da is not None:
+        da.copy_(torch.from_numpy(dh.sum(axis=0)))
+
+
+def mlp_tp_fc2_backward_weight(H, H_lo, dY, T, h, f, t, dB, db, ws, stream=None):
+    hh = _np(H) + (_np(H_lo) if H_lo is not None else 0.0)
+    dB.copy_(torch.from_numpy(hh.T @ _np(dY)))
+    if db is not None:
+        db.copy_(torch.from_numpy(_np(dY).sum(axis=0)))
+
+
+def mlp_tp_fc1_backward_data(dH, dH_lo, A, T, h, f, t, dX, ws, stream=None):
+    dh = _np(dH) + (_np(dH_lo) if dH_lo is not None else 0.0)
+    dX.copy_(torch.from_numpy(dh @ _np(A).T))
+
+
+def mlp_tp_fc1_backward_weight(X, dH, dH_lo, T, h, f, t, dA, ws, stream=None):
+    dh = _np(dH) + (_np(dH_lo) if dH_lo is not None else 0.0)
+    dA.copy_(torch.from_numpy(np.asarray(_np(X)).T @ dh))
