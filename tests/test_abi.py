@@ -117,3 +117,46 @@ def test_split_flags_are_validated(lib):
     st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, 1024, 2, 7, FAKE, FAKE, FAKE, FAKE,
                             FAKE * 2, 1 << 30, None)
     assert st == 1 and "split" in binding.mlp_tp_last_error()
+
+
+C_CLIENT = r"""
+/* A plain C99 client of the library: no CUDA headers, no torch. */
+#include <stdio.h>
+#include <string.h>
+#include "mlp_tp.h"
+
+int main(void) {
+  size_t n = mlp_tp_workspace_bytes(64, 256, 1024, 2);
+  if (n == 0) return 1;
+  if (mlp_tp_workspace_bytes(64, 256, 1000, 3) != 0) return 2;          /* f not divisible by t */
+  if (strcmp(mlp_tp_status_string(MLP_ERR_MISALIGNED), "MLP_ERR_MISALIGNED") != 0) return 3;
+  /* NULL X is refused on the host, before any device work */
+  mlp_status_t st = mlp_tp_fc1_forward(NULL, (void*)0x100000, (void*)0x100000, 64, 256, 1024, 2,
+                                       (void*)0x100000, (void*)0x100000, (void*)0x100000,
+                                       (void*)0x200000, (size_t)1 << 30, NULL);
+  if (st != MLP_ERR_INVALID_ARG || strstr(mlp_tp_last_error(), "X") == NULL) return 4;
+  printf("%zu\n", n);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """The header compiles as C99 and a C program links the library and
+    calls it (host-side entry points only: no GPU here)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(binding.LIB_PATH)
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+           "-o", str(exe), "-L", libdir, "-l:" + os.path.basename(binding.LIB_PATH), "-Wl,-rpath," + libdir]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    assert int(run.stdout.strip()) == binding.workspace_bytes(64, 256, 1024, 2)
