@@ -49,7 +49,13 @@
  *    a workspace must be ordered on one stream.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point except mlp_tp_check synchronises, and
- *    none allocates or frees memory.
+ *    none allocates or frees memory.  The enqueued work is kernel launches
+ *    and asynchronous memsets only, so a sequence of calls can be captured
+ *    into a CUDA graph and replayed (after one uncaptured call per shape,
+ *    which sets the kernels' shared-memory limits); a replay reads the
+ *    buffers' current contents.
+ *  - Results are reproducible bit for bit for a given GPU model, shape and
+ *    t: every reduction runs in a fixed order.
  *  - Arguments are validated on the host before anything is launched; on any
  *    error nothing is enqueued.  Errors raised by the CUDA runtime when
  *    launching map to MLP_ERR_CUDA.  Faults found by the kernels themselves
@@ -80,8 +86,10 @@ typedef enum {
 
 /* Bytes of workspace needed by every entry point below for this shape
  * (the maximum over all of them): a 256-byte status header, the dH pair
- * used by mlp_tp_backward, and fp32 column-sum partials.  Returns 0 for an
- * invalid shape. */
+ * used by mlp_tp_backward, fp32 column-sum partials, and fp32 scratch for
+ * output tiles whose K loop is split into pieces (the shard sums of a
+ * partial last wave, or the weight gradients when they have fewer tiles
+ * than the GPU has CTA pairs).  Returns 0 for an invalid shape. */
 size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
 
 /* Split flags of the composite calls: which second-layer products also use
