@@ -81,7 +81,9 @@ typedef enum {
   MLP_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < mlp_tp_workspace_bytes(...) */
   MLP_ERR_UNSUPPORTED_DEVICE = 5,  /* current device is not sm_100, or none */
   MLP_ERR_CUDA = 6,                /* the CUDA runtime reported an error */
-  MLP_ERR_TIMEOUT = 7              /* a kernel's bounded wait ran out (mlp_tp_check) */
+  MLP_ERR_TIMEOUT = 7,             /* a kernel's bounded wait ran out (mlp_tp_check) */
+  MLP_ERR_BOUNDS = 8               /* bounds-checking build only: an index fell outside its
+                                      buffer; the access was skipped (mlp_tp_check) */
 } mlp_status_t;
 
 /* Bytes of workspace needed by every entry point below for this shape
@@ -231,8 +233,10 @@ mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, int64_t h, 
 
 /* Synchronises `stream`, then reads and clears the device status word in
  * `ws`.  Returns MLP_OK, MLP_ERR_TIMEOUT (a kernel's bounded wait ran out;
- * its outputs are undefined, the CUDA context stays usable) or MLP_ERR_CUDA
- * (the stream reported an error). */
+ * its outputs are undefined, the CUDA context stays usable), MLP_ERR_BOUNDS
+ * (only from a library built with -DMLPTP_BOUNDS_CHECK: a plain global
+ * access outside its buffer was found and skipped) or MLP_ERR_CUDA (the
+ * stream reported an error). */
 mlp_status_t mlp_tp_check(void* ws, void* stream);
 
 /* Static, NUL-terminated name of a status code. */

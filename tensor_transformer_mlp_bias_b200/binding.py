@@ -25,6 +25,7 @@ STATUS = {
     5: "MLP_ERR_UNSUPPORTED_DEVICE",
     6: "MLP_ERR_CUDA",
     7: "MLP_ERR_TIMEOUT",
+    8: "MLP_ERR_BOUNDS",
 }
 
 # name -> argument ctypes, in header order

@@ -40,18 +40,23 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Builds the library; returns its path.  `defines` (e.g.
+    ["MLPTP_BOUNDS_CHECK"]) and `out` build a variant at another path (always
+    rebuilt) instead of the in-tree library."""
+    target = out or OUT
+    if out is None and not defines and not force and up_to_date():
         return OUT
-    tmp = OUT + ".tmp"
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp, SRC]
+    tmp = target + ".tmp"
+    cmd = ([nvcc()] + NVCC_FLAGS + ["-D" + d for d in defines] + (["-Xptxas", "-v"] if verbose else []) +
+           ["-o", tmp, SRC])
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

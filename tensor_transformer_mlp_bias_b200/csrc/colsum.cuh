@@ -15,13 +15,16 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "gemm.cuh"  // index_ok, the bounds-checking build's index check
+
 namespace mlptp {
 
 constexpr int COLSUM_ROWS_PER_CHUNK = 256;
 constexpr int COLSUM_COLS_PER_BLOCK = 32 * 8;
 
 __global__ void __launch_bounds__(256) colsum_partial(const __nv_bfloat16* __restrict__ m, int R, int C,
-                                                      float* __restrict__ partial) {
+                                                      float* __restrict__ partial, long long partial_elems,
+                                                      unsigned int* status) {
   __shared__ float red[8][32][9];
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int c0 = (blockIdx.x * 32 + tx) * 8;
@@ -33,6 +36,7 @@ __global__ void __launch_bounds__(256) colsum_partial(const __nv_bfloat16* __res
   if (c0 < C) {
     const __nv_bfloat16* base = m + c0;
     for (int r = r_begin + ty; r < r_end; r += 8) {
+      if (!index_ok(static_cast<long long>(r) * C + c0 + 7, static_cast<long long>(R) * C, status, 0x506u)) break;
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * C));
       const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -56,16 +60,21 @@ __global__ void __launch_bounds__(256) colsum_partial(const __nv_bfloat16* __res
       for (int y = 1; y < 8; ++y) s += red[y][tx][e];
       out[e] = s;
     }
-    float4* dst = reinterpret_cast<float4*>(partial + static_cast<size_t>(blockIdx.y) * C + c0);
-    dst[0] = make_float4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+    const long long pi = static_cast<long long>(blockIdx.y) * C + c0;
+    if (index_ok(pi + 7, partial_elems, status, 0x507u)) {
+      float4* dst = reinterpret_cast<float4*>(partial + pi);
+      dst[0] = make_float4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+    }
   }
 }
 
 __global__ void __launch_bounds__(256) colsum_final(const float* __restrict__ partial, int chunks, int C,
-                                                    __nv_bfloat16* __restrict__ out) {
+                                                    __nv_bfloat16* __restrict__ out, long long partial_elems,
+                                                    unsigned int* status) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= C) return;
+  if (!index_ok(static_cast<long long>(chunks - 1) * C + c, partial_elems, status, 0x508u)) return;
   float s = 0.0f;
   for (int k = 0; k < chunks; ++k) s += partial[static_cast<size_t>(k) * C + c];
   out[c] = __float2bfloat16_rn(s);

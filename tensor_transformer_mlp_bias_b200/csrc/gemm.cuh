@@ -123,6 +123,31 @@ struct TileCfg {
 };
 
 constexpr unsigned int STATUS_TIMEOUT = 7u;
+constexpr unsigned int STATUS_BOUNDS = 8u;
+
+// Bounds-checking build (compiled with -DMLPTP_BOUNDS_CHECK): every plain
+// global access that does not go through a tensor map checks the last
+// element it touches against its buffer's element count.  A bad index
+// records status 8 and the access site in the status word and skips the
+// access (no trap, no device assert).  In the normal build the check
+// compiles away.
+__device__ __forceinline__ bool index_ok(long long last, long long n, unsigned int* status, unsigned int site) {
+#ifdef MLPTP_BOUNDS_CHECK
+  if (last < 0 || last >= n) {
+    if (status != nullptr) {  // the allocation-free path has no status word
+      atomicCAS(status, 0u, STATUS_BOUNDS);
+      atomicCAS(status + 1, 0u, site);
+    }
+    return false;
+  }
+#else
+  (void)last;
+  (void)n;
+  (void)status;
+  (void)site;
+#endif
+  return true;
+}
 
 struct GemmParams {
   int M, N;
@@ -135,6 +160,7 @@ struct GemmParams {
   // tail_scratch and a separate kernel adds the pieces of a tile in order.
   int full_tiles, tail_split, kb_split, num_work;
   float* tail_scratch;    // [pieces][TILE_M][TILE_N] fp32
+  long long scratch_elems;  // floats in tail_scratch (bounds-checking build)
   int parts;              // 1, or 2 when an operand is a bf16 (hi, lo) pair
   int kblocks_per_shard;  // BK-wide K slices per segment and part
   int m_blocks, n_blocks, num_tiles, group_m;
@@ -142,6 +168,7 @@ struct GemmParams {
   __nv_bfloat16* out1;        // H_lo (EPI_BIAS_GELU) | dH_lo (EPI_GELU_GRAD)
   float* out_f32;             // Z (EPI_BIAS_GELU)
   float* colsum;              // [row blocks*4, N] column sums of dH (EPI_GELU_GRAD), may be null
+  long long colsum_elems;     // floats in colsum (bounds-checking build)
   const __nv_bfloat16* bias;  // a (EPI_BIAS_GELU) or b (EPI_SHARD_SUM), may be null for the latter
   const float* aux;           // Z (EPI_GELU_GRAD)
   unsigned int* status;       // device status word pair in the workspace
@@ -288,18 +315,6 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&d
   uint4 w[4];
   load_bf16x32_raw(src, w);
   widen_bf16x32(w, dst);
-}
-
-__device__ __forceinline__ void load_f32x32(const float* src, float (&dst)[32]) {
-  const float4* s = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int v = 0; v < 8; ++v) {
-    const float4 w = __ldg(s + v);
-    dst[4 * v] = w.x;
-    dst[4 * v + 1] = w.y;
-    dst[4 * v + 2] = w.z;
-    dst[4 * v + 3] = w.w;
-  }
 }
 
 // Row `r` (this lane) of a 32x32 bf16 staging tile: 64-byte rows, 16-byte
@@ -728,14 +743,17 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             }
             if (p.colsum != nullptr) {
               const float cs = warp_column_sums(dh);
-              p.colsum[static_cast<size_t>(row_block * 4 + q) * p.N + col + lane] = cs;
+              const long long ci = static_cast<long long>(row_block * 4 + q) * p.N + col + lane;
+              if (index_ok(ci, p.colsum_elems, p.status, 0x501u)) p.colsum[ci] = cs;
             }
           } else if constexpr (EPI == EPI_STORE) {
             if (it.piece >= 0) {
               // one K piece of a split tile: its fp32 sum goes to the scratch
-              float4* d4 = reinterpret_cast<float4*>(
-                  p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
-                  static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS + c * 32);
+              const long long si = static_cast<long long>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
+                                   static_cast<long long>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS +
+                                   c * 32;
+              if (!index_ok(si + 31, p.scratch_elems, p.status, 0x502u)) continue;
+              float4* d4 = reinterpret_cast<float4*>(p.tail_scratch + si);
 #pragma unroll
               for (int j = 0; j < 8; ++j)
                 d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
@@ -762,13 +780,16 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             }
             if (s == it.s_end - 1 && it.piece >= 0) {
               // one piece of a split tile: its fp32 sum goes to the scratch
-              float* dst = p.tail_scratch + static_cast<size_t>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
-                           static_cast<size_t>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS + c * 32;
-              float4* d4 = reinterpret_cast<float4*>(dst);
+              const long long si = static_cast<long long>(it.piece) * (Cfg::TILE_M * Cfg::TILE_N) +
+                                   static_cast<long long>(rank * BM + q * 32 + lane) * Cfg::TILE_N + slice * SLICE_COLS +
+                                   c * 32;
+              if (index_ok(si + 31, p.scratch_elems, p.status, 0x503u)) {
+                float4* d4 = reinterpret_cast<float4*>(p.tail_scratch + si);
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                d4[j] = make_float4(sum[c * 32 + 4 * j], sum[c * 32 + 4 * j + 1], sum[c * 32 + 4 * j + 2],
-                                    sum[c * 32 + 4 * j + 3]);
+                for (int j = 0; j < 8; ++j)
+                  d4[j] = make_float4(sum[c * 32 + 4 * j], sum[c * 32 + 4 * j + 1], sum[c * 32 + 4 * j + 2],
+                                      sum[c * 32 + 4 * j + 3]);
+              }
             } else if (s == it.s_end - 1) {
               float bias[32];
               if (p.bias != nullptr) {
@@ -845,9 +866,10 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const GemmParams p, i
   if (row >= p.M || col >= p.N) return;
   float acc[8];
   for (int part = 0; part < split; ++part) {
-    const float4* src = reinterpret_cast<const float4*>(
-        p.tail_scratch + static_cast<size_t>(t_local * split + part) * (TILE_M * TILE_N) +
-        static_cast<size_t>(r) * TILE_N + c8);
+    const long long si = static_cast<long long>(t_local * split + part) * (TILE_M * TILE_N) +
+                         static_cast<long long>(r) * TILE_N + c8;
+    if (!index_ok(si + 7, p.scratch_elems, p.status, 0x504u)) return;
+    const float4* src = reinterpret_cast<const float4*>(p.tail_scratch + si);
     const float4 v0 = src[0], v1 = src[1];
     const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
@@ -871,7 +893,9 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const GemmParams p, i
   o.y = pack_bf16x2(acc[2] + bias[2], acc[3] + bias[3]);
   o.z = pack_bf16x2(acc[4] + bias[4], acc[5] + bias[5]);
   o.w = pack_bf16x2(acc[6] + bias[6], acc[7] + bias[7]);
-  *reinterpret_cast<uint4*>(p.out0 + static_cast<size_t>(row) * p.N + col) = o;
+  const long long oi = static_cast<long long>(row) * p.N + col;
+  if (index_ok(oi + 7, static_cast<long long>(p.M) * p.N, p.status, 0x505u))
+    *reinterpret_cast<uint4*>(p.out0 + oi) = o;
 }
 
 }  // namespace mlptp

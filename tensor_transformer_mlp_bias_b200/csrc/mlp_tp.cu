@@ -422,6 +422,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
       p.kb_split = best_k;
       p.full_tiles = 0;
       p.tail_scratch = g.tail_scratch;
+      p.scratch_elems = static_cast<long long>(g.tail_bytes / sizeof(float));
     }
   }
   if (EPI == EPI_SHARD_SUM && p.shards > 1 && capacity > 0) {
@@ -442,6 +443,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
         p.full_tiles = p.num_tiles - tail;
         p.tail_split = best_k;
         p.tail_scratch = g.tail_scratch;
+        p.scratch_elems = static_cast<long long>(g.tail_bytes / sizeof(float));
       }
     }
   }
@@ -480,16 +482,21 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   return MLP_OK;
 }
 
-mlp_status_t launch_colsum_final(const float* partial, int chunks, int64_t C, void* out, cudaStream_t stream) {
-  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(partial, chunks, static_cast<int>(C),
-                                                                           static_cast<__nv_bfloat16*>(out));
+// `partial_elems` is the size of the partial-sum buffer and `status` the
+// workspace status word (NULL: none); both serve the bounds-checking build.
+mlp_status_t launch_colsum_final(const float* partial, int chunks, int64_t C, void* out, cudaStream_t stream,
+                                 size_t partial_elems, unsigned int* status) {
+  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(
+      partial, chunks, static_cast<int>(C), static_cast<__nv_bfloat16*>(out), static_cast<long long>(partial_elems),
+      status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "colsum_final");
   g_launches.fetch_add(1);
   return MLP_OK;
 }
 
-mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float* partial, cudaStream_t stream) {
+mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float* partial, cudaStream_t stream,
+                           size_t partial_elems, unsigned int* status) {
   if (R == 0) {
     cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(C) * 2, stream);
     return e == cudaSuccess ? MLP_OK : cuda_fail(e, "cudaMemsetAsync(bias gradient)");
@@ -497,11 +504,12 @@ mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float
   const int chunks = static_cast<int>(colsum_chunks(R));
   dim3 grid1(static_cast<unsigned>((C + COLSUM_COLS_PER_BLOCK - 1) / COLSUM_COLS_PER_BLOCK), chunks);
   colsum_partial<<<grid1, dim3(32, 8), 0, stream>>>(static_cast<const __nv_bfloat16*>(m), static_cast<int>(R),
-                                                    static_cast<int>(C), partial);
+                                                    static_cast<int>(C), partial,
+                                                    static_cast<long long>(partial_elems), status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "colsum_partial");
   g_launches.fetch_add(1);
-  return launch_colsum_final(partial, chunks, C, out, stream);
+  return launch_colsum_final(partial, chunks, C, out, stream, partial_elems, status);
 }
 
 mlp_status_t zero_fill(void* p, size_t bytes, cudaStream_t s, const char* what) {
@@ -571,6 +579,7 @@ mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, co
   p.out1 = static_cast<__nv_bfloat16*>(dH_lo);
   p.aux = static_cast<const float*>(Z);
   p.colsum = da != nullptr ? partials(ws, s) : nullptr;
+  p.colsum_elems = static_cast<long long>(partial_bytes(s) / sizeof(float));
   GemmDesc g{one(dY, false), one(B, false), s.T, s.f, s.h, 1, 1};
   // 16 epilogue warps when K = h is short enough for the epilogue (loads of
   // Z, g'(Z), the dH pair, column sums) to outlast the mainloop of a tile:
@@ -580,7 +589,8 @@ mlp_status_t fc2_backward_data(const Shape& s, const void* dY, const void* B, co
           ? launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 16>(g, p, L, "row-parallel backward data (dH, da)")
           : launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 8>(g, p, L, "row-parallel backward data (dH, da)");
   if (st != MLP_OK || da == nullptr) return st;
-  return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream);
+  return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream,
+                             partial_bytes(s) / sizeof(float), static_cast<unsigned int*>(ws));
 }
 
 mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* H_lo, const void* dY, void* dB, void* db,
@@ -595,7 +605,8 @@ mlp_status_t fc2_backward_weight(const Shape& s, const void* H, const void* H_lo
     st = launch_gemm<true, true, EPI_STORE, kWideTN, kPair, 8, kDualA>(g, p, L, "row-parallel weight gradient (dB)");
   }
   if (st != MLP_OK || db == nullptr) return st;
-  return launch_colsum(dY, s.T, s.h, db, partials(ws, s), L.stream);
+  return launch_colsum(dY, s.T, s.h, db, partials(ws, s), L.stream, partial_bytes(s) / sizeof(float),
+                       static_cast<unsigned int*>(ws));
 }
 
 mlp_status_t fc1_backward_data(const Shape& s, const void* dH, const void* dH_lo, const void* A, void* dX, void* ws,
@@ -823,6 +834,8 @@ mlp_status_t mlp_tp_check(void* ws, void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace status word");
   if (word[0] == STATUS_TIMEOUT)
     return fail(MLP_ERR_TIMEOUT, "a kernel wait ran out of its budget (site 0x%x)", word[1]);
+  if (word[0] == STATUS_BOUNDS)
+    return fail(MLP_ERR_BOUNDS, "an index fell outside its buffer (site 0x%x; bounds-checking build)", word[1]);
   return fail(MLP_ERR_CUDA, "device status word holds unknown code %u", word[0]);
 }
 
@@ -835,6 +848,7 @@ const char* mlp_tp_status_string(mlp_status_t status) {
     case MLP_ERR_WORKSPACE_TOO_SMALL: return "MLP_ERR_WORKSPACE_TOO_SMALL";
     case MLP_ERR_UNSUPPORTED_DEVICE: return "MLP_ERR_UNSUPPORTED_DEVICE";
     case MLP_ERR_CUDA: return "MLP_ERR_CUDA";
+    case MLP_ERR_BOUNDS: return "MLP_ERR_BOUNDS";
     case MLP_ERR_TIMEOUT: return "MLP_ERR_TIMEOUT";
   }
   return "MLP_ERR_UNKNOWN";
@@ -898,5 +912,5 @@ extern "C" mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, 
   if ((st = noalloc_scratch(dev, &scratch)) != MLP_OK) return st;
   // Pass 1 overwrites every partial it reads back in pass 2, so nothing left
   // in the array by an earlier call is ever used.
-  return launch_colsum(dY, T, h, db, scratch, static_cast<cudaStream_t>(stream));
+  return launch_colsum(dY, T, h, db, scratch, static_cast<cudaStream_t>(stream), NOALLOC_MAX_PARTIALS, nullptr);
 }

@@ -1,0 +1,56 @@
+"""The bounds-checking build (-DMLPTP_BOUNDS_CHECK) on the GPU.
+
+In that build every plain global access that does not go through a tensor
+map (the column-sum partials, the fp32 pieces of split tiles and their
+reduce, the bias-gradient column sums) checks its index against its buffer
+and reports MLP_ERR_BOUNDS from mlp_tp_check instead of touching memory
+outside it.  It stands in for a memory checker, which this machine does not
+offer.  The shapes below reach every checked site: split shard-sum tails,
+K-split weight gradients, ragged tiles, da and db.  They must pass with a
+clean status word and meet the parity bar.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from tensor_transformer_mlp_bias_b200 import build
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r"""
+import sys
+sys.path.insert(0, sys.argv[1])
+from tensor_transformer_mlp_bias_b200 import binding
+binding.LIB_PATH = sys.argv[2]
+from oracle import mlp_oracle as oracle
+from tensor_transformer_mlp_bias_b200 import block, inputs
+from tests.parity_util import assert_close, to_gpu
+shapes = [(333, 320, 1280, 5, 0), (1024, 256, 1024, 2, 0), (2048, 128, 512, 4, 3), (1, 64, 128, 2, 0),
+          (257, 512, 768, 3, 3)]
+for T, h, f, t, split in shapes:
+    inp = inputs.make_custom(T, h, f, seed=T + f)
+    out = block.forward_backward(to_gpu(inp), t, split=split)  # mlp_tp_check raises on MLP_ERR_BOUNDS
+    ref = oracle.full(inp)
+    for k in ("Y", "dX", "dA", "da", "dB", "db"):
+        assert_close(k, out[k], ref[k])
+import torch
+T, h = 4096, 1024
+dY = to_gpu(inputs.make_custom(T, h, 256, seed=3))["dY"]
+db = torch.empty(h, dtype=torch.bfloat16, device="cuda")  # h elements, as the call writes
+binding.mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db)
+torch.cuda.synchronize()
+assert_close("db (allocation-free)", db, dY.double().sum(0).cpu().numpy())
+print("bounds-checked build: clean")
+"""
+
+
+def test_bounds_checked_build_is_clean(tmp_path):
+    lib = build.build(defines=["MLPTP_BOUNDS_CHECK"], out=str(tmp_path / "libmlptp_bounds.so"))
+    res = subprocess.run([sys.executable, "-c", CHILD, ROOT, lib], capture_output=True, text=True, timeout=600,
+                         cwd=ROOT)
+    assert res.returncode == 0, res.stdout[-2000:] + res.stderr[-4000:]
+    assert "clean" in res.stdout
