@@ -130,18 +130,34 @@ size_t tail_pieces_capacity(const Shape& s) {
   return n < TAIL_MAX_PIECES ? n : TAIL_MAX_PIECES;
 }
 size_t tail_offset(const Shape& s) { return partial_offset(s) + partial_bytes(s); }
-// K pieces of the weight-gradient GEMMs when they have fewer tiles than CTA
-// pairs: at most KSPLIT_MAX_PIECES pieces of 256x512 fp32, and no more than
-// one piece per 8 K slices of every tile.
+// K pieces of the weight-gradient GEMMs.
+//  - Fewer tiles than CTA pairs: at most KSPLIT_MAX_PIECES pieces of 256x512
+//    fp32, and no more than one piece per 8 K slices of every tile.
+//  - Long token axes: a weight gradient's K loop runs over the T tokens, and
+//    one fp32 TMEM accumulator takes at most kWgradMaxAdds tensor-core
+//    additions (4 per 64-token K slice and product; both halves of the pair
+//    count): 16384 tokens.  Measured on B200: dB over 65536 tokens in one
+//    accumulator reached 1.14 of the parity bar, while 16384 tokens pass
+//    with a wide margin; the tensor core's accumulation is not round-to-
+//    nearest fp32, and its error grows with the number of additions.  Longer
+//    K loops are cut into ceil(T / 16384) pieces or more, which the reduce
+//    pass adds in fp32 in K order.
 constexpr size_t KSPLIT_MAX_PIECES = 128;
 constexpr size_t KSPLIT_PIECE_BYTES = static_cast<size_t>(TileShape::TILE_M) * 512 * sizeof(float);
+constexpr int64_t kWgradMaxAdds = 2048;
+int64_t wgrad_min_pieces(int64_t T) {
+  const int64_t adds = 8 * ((T + BK - 1) / BK);  // 4 per slice, times the 2 halves of the pair
+  return (adds + kWgradMaxAdds - 1) / kWgradMaxAdds;
+}
 size_t ksplit_bytes(const Shape& s) {
   const size_t kb = 2 * static_cast<size_t>((s.T + BK - 1) / BK);  // two parts (hi, lo)
   const size_t per_tile = kb / 8;
   const size_t tiles_dA = static_cast<size_t>((s.h + 255) / 256) * static_cast<size_t>((s.f + 511) / 512);
   const size_t tiles_dB = static_cast<size_t>((s.f + 255) / 256) * static_cast<size_t>((s.h + 511) / 512);
   const size_t tiles = tiles_dA > tiles_dB ? tiles_dA : tiles_dB;
-  const size_t pieces = tiles * per_tile < KSPLIT_MAX_PIECES ? tiles * per_tile : KSPLIT_MAX_PIECES;
+  size_t pieces = tiles * per_tile < KSPLIT_MAX_PIECES ? tiles * per_tile : KSPLIT_MAX_PIECES;
+  const size_t min_k = static_cast<size_t>(wgrad_min_pieces(s.T));
+  if (min_k > 1 && tiles * min_k > pieces) pieces = tiles * min_k;
   return pieces * KSPLIT_PIECE_BYTES;
 }
 size_t split_scratch_bytes(const Shape& s) {
@@ -407,11 +423,17 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   const size_t capacity = g.tail_scratch != nullptr ? g.tail_bytes / piece_bytes : 0;
   const int kb_per_unit = p.parts * p.kblocks_per_shard;  // slices per shard
   auto rounds = [&](long long items) { return static_cast<double>((items + max_clusters - 1) / max_clusters); };
-  if (EPI == EPI_STORE && p.num_tiles < max_clusters && capacity >= 2) {
+  // weight gradients: at least enough pieces to keep each accumulator within
+  // kWgradMaxAdds additions (long token axes)
+  const int64_t adds_per_unit = static_cast<int64_t>(kb_per_unit) * (BK / 16) * (DUAL ? 2 : 1);
+  const int min_k = EPI == EPI_STORE ? static_cast<int>((adds_per_unit + kWgradMaxAdds - 1) / kWgradMaxAdds) : 1;
+  if (min_k > 1 && static_cast<size_t>(min_k) * p.num_tiles > capacity)
+    return fail(MLP_ERR_WORKSPACE_TOO_SMALL, "%s: %d K pieces per tile do not fit the split scratch", name, min_k);
+  if (EPI == EPI_STORE && (p.num_tiles < max_clusters || min_k > 1) && capacity >= 2) {
     const double U = kb_per_unit;
-    int best_k = 1;
-    double best = U;
-    for (int k = 2; k <= kb_per_unit / 8 && static_cast<size_t>(k) * p.num_tiles <= capacity; ++k) {
+    int best_k = min_k;
+    double best = min_k == 1 ? U : rounds(static_cast<long long>(p.num_tiles) * min_k) * (U / min_k + kPieceOverheadSlices);
+    for (int k = min_k + 1; k <= kb_per_unit / 8 && static_cast<size_t>(k) * p.num_tiles <= capacity; ++k) {
       const double cost = rounds(static_cast<long long>(p.num_tiles) * k) * (U / k + kPieceOverheadSlices);
       if (cost < best - 1e-9) {
         best = cost;

@@ -6,8 +6,9 @@ reduce, the bias-gradient column sums) checks its index against its buffer
 and reports MLP_ERR_BOUNDS from mlp_tp_check instead of touching memory
 outside it.  It stands in for a memory checker, which this machine does not
 offer.  The shapes below reach every checked site: split shard-sum tails,
-K-split weight gradients, ragged tiles, da and db.  They must pass with a
-clean status word and meet the parity bar.
+K-split weight gradients, ragged tiles, da and db, and a batch whose [T, f]
+tensors hold more than 2^31 elements.  They must pass with a clean status
+word and meet the parity bar.
 """
 import os
 import subprocess
@@ -37,7 +38,25 @@ for T, h, f, t, split in shapes:
     ref = oracle.full(inp)
     for k in ("Y", "dX", "dA", "da", "dB", "db"):
         assert_close(k, out[k], ref[k])
+import numpy as np
 import torch
+# T*f above 2^31 elements: every plain index must be 64-bit (sampled oracle)
+T, h, f, t = 65536, 1024, 33280, 8
+inp = inputs.make_custom(T, h, f, seed=71)
+out = block.forward_backward(to_gpu(inp), t)
+rows = np.array([0, 1, 30000, 65535])
+cols = np.array([0, 5, 20000, 33279])
+sr = oracle.sample_rows(inp, rows)
+sc = oracle.sample_ffn(inp, cols)
+r = torch.as_tensor(rows, device="cuda")
+c = torch.as_tensor(cols, device="cuda")
+assert_close("Y rows", out["Y"][r], sr["Y"])
+assert_close("dX rows", out["dX"][r], sr["dX"])
+assert_close("dA cols", out["dA"][:, c], sc["dA"])
+assert_close("dB rows", out["dB"][c, :], sc["dB"])
+assert_close("da cols", out["da"][c], sc["da"])
+del out, inp
+torch.cuda.empty_cache()
 T, h = 4096, 1024
 dY = to_gpu(inputs.make_custom(T, h, 256, seed=3))["dY"]
 db = torch.empty(h, dtype=torch.bfloat16, device="cuda")  # h elements, as the call writes
