@@ -547,6 +547,8 @@ def main():
                        tensor_flops_per_step=2.0 * T * h * f * sum(products.values())),
         "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_DENSE_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * value / world / float(peaks.get("bf16_tflops", 1713.1)),
+        # cuBLAS looped for seconds under the power cap, like this 200-step region
+        "pct_of_measured_sustained_bf16_peak": 100.0 * value / world / peak_sustained,
         "stage_ms": stage_ms,
         "per_t": dict(sorted(per_t.items(), key=lambda kv: int(kv[0]))),
         "roofline": roofline,
