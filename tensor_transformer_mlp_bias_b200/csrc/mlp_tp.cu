@@ -508,7 +508,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
 // workspace status word (NULL: none); both serve the bounds-checking build.
 mlp_status_t launch_colsum_final(const float* partial, int chunks, int64_t C, void* out, cudaStream_t stream,
                                  size_t partial_elems, unsigned int* status) {
-  colsum_final<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(
+  colsum_final<<<static_cast<unsigned>((C + 31) / 32), dim3(32, 8), 0, stream>>>(
       partial, chunks, static_cast<int>(C), static_cast<__nv_bfloat16*>(out), static_cast<long long>(partial_elems),
       status);
   cudaError_t e = cudaGetLastError();
@@ -525,7 +525,7 @@ mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float
   }
   const int chunks = static_cast<int>(colsum_chunks(R));
   dim3 grid1(static_cast<unsigned>((C + COLSUM_COLS_PER_BLOCK - 1) / COLSUM_COLS_PER_BLOCK), chunks);
-  colsum_partial<<<grid1, dim3(32, 8), 0, stream>>>(static_cast<const __nv_bfloat16*>(m), static_cast<int>(R),
+  colsum_partial<<<grid1, dim3(32, COLSUM_PHASES), 0, stream>>>(static_cast<const __nv_bfloat16*>(m), static_cast<int>(R),
                                                     static_cast<int>(C), partial,
                                                     static_cast<long long>(partial_elems), status);
   cudaError_t e = cudaGetLastError();
