@@ -1,5 +1,5 @@
 """Cross-GPU orchestration of the block (tensor_transformer_mlp_bias_b200.tp)
-as two gloo ranks on the CPU.
+as two and four gloo ranks on the CPU.
 
 Each rank holds one shard (its column block of A and a, its row block of B)
 and runs the stage calls through the fp64 stand-in in tests/tp_cpu_ops.py;
@@ -84,6 +84,14 @@ def _run(world, shape, sp, split):
 def test_two_ranks_match_the_unsharded_block(sp, split):
     res = _run(2, (64, 128, 256), sp, split)
     assert set(res) == {0, 1}
+    for rank, errs in res.items():
+        for k, e in errs.items():
+            assert e < 1e-12, (rank, k, e)
+
+
+def test_four_ranks_sequence_parallel_match_the_unsharded_block():
+    res = _run(4, (64, 128, 512), True, 0)
+    assert set(res) == {0, 1, 2, 3}
     for rank, errs in res.items():
         for k, e in errs.items():
             assert e < 1e-12, (rank, k, e)
