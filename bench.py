@@ -20,6 +20,24 @@ the device and copies only X, dY in and Y, dX out), `roofline` for the dominant 
 oracle timed on this host's cores on a bounded sample), the GPU clocks seen
 during the timed region and the number of library kernel launches in it.
 
+Precision mode.  The library's default (accurate) mode takes Y and dX over
+both halves of the bf16 activation pair; the fast mode takes them from the
+high half only.  `--mode auto` times the fast mode on the workloads where its
+GPU parity test meets the bar (tiny, GPT-2-medium, h4096, 175B-class) and the
+accurate mode otherwise; the line says which (`precision_mode`), and with the
+fast mode it also times the accurate mode over as many steps (`accurate`).
+
+Roofline.  `roofline.achieved` is the dominant stage's algorithmic FLOPs
+(2·T·h·f per GEMM) over its CUDA-event time; `executed_tflops` counts every
+tensor-core product it runs (the weight gradients run two per GEMM).  The
+peak is the measured burst bf16 figure unless the SM clock sampled while the
+stages were timed sat clearly below its maximum (median < 0.97·max), when it
+is the measured sustained figure.
+
+`steady` times the same step loop for at least two seconds, long enough for
+the clock to settle under the power cap; both it and the headline report the
+median SM clock and ms-per-step × MHz.
+
 --impl reference times the fp64 CPU oracle itself as the reference arm.
 """
 from __future__ import annotations
@@ -53,9 +71,57 @@ STAGE_KERNEL = {
     "fc1_backward_data": "dX=Σ_i dH_i·A_iᵀ (GEMM, shard-sum epilogue)",
     "fc1_backward_weight": "dA=Xᵀ·(dH+dH_lo) (GEMM over both halves)",
 }
-# tensor-core products each stage's GEMM runs, in units of 2·T·h·f
+# tensor-core products each stage's GEMM runs in the fast mode, in units of 2·T·h·f
 STAGE_PRODUCTS = {"fc1_forward": 1, "fc2_forward": 1, "fc2_backward_data": 1, "fc2_backward_weight": 2,
                   "fc1_backward_data": 1, "fc1_backward_weight": 2}
+MODES = {"accurate": 0, "fast": 3}
+# workloads whose GPU parity test runs the fast mode and meets the bar
+FAST_MODE_PARITY = ("tiny", "gpt2-medium", "h4096", "175b-class")
+STEADY_SECONDS = 2.0
+
+
+def stage_products(mode):
+    """Tensor-core products per stage for a precision mode (flags 1 and 2
+    drop the low half from the Y and dX GEMMs)."""
+    p = dict(STAGE_PRODUCTS)
+    p["fc2_forward"] += 0 if mode & 1 else 1
+    p["fc1_backward_data"] += 0 if mode & 2 else 1
+    return p
+
+
+def pick_mode(arg, wl_name):
+    if arg == "auto":
+        return "fast" if wl_name in FAST_MODE_PARITY else "accurate"
+    return arg
+
+
+def roofline_entry(stage_ms, mode, T, h, f, clocks, peaks, peak_src):
+    """Roofline of the dominant (longest) stage.  achieved = its algorithmic
+    FLOPs (one GEMM, 2·T·h·f) per launch over its mean CUDA-event time;
+    frac = achieved / peak.  The peak is the measured burst bf16 figure
+    unless the SM clock sampled while the stages were timed sat below 0.97 of
+    its maximum, then the measured sustained one."""
+    products = stage_products(mode)
+    dom = max(STAGES, key=lambda k: stage_ms[k])
+    unit = 2.0 * T * h * f
+    secs = stage_ms[dom] * 1e-3
+    achieved = unit / secs / 1e12
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    settled = bool(mhz and mx and mhz < 0.97 * mx)
+    peak = sustained if settled else burst
+    kind = ("bf16_tflops_sustained (SM clock median %.0f of %.0f MHz while the stages were timed)" % (mhz, mx)
+            if settled else "bf16_tflops (burst; SM clock median %s of %s MHz while the stages were timed)"
+            % (mhz, mx))
+    return {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved, "peak": peak,
+            "unit": UNIT, "frac": achieved / peak, "peak_source": f"{peak_src} {kind}",
+            "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+            "algorithmic_flops_per_launch": unit, "avg_launch_ms": stage_ms[dom],
+            "executed_tensor_products": products[dom],
+            "executed_tflops": unit * products[dom] / secs / 1e12,
+            "executed_frac_of_peak": unit * products[dom] / secs / 1e12 / peak,
+            "stage_clocks": clocks}
 
 
 # ---------------------------------------------------------------- helpers
@@ -93,15 +159,20 @@ def reduce_max_sum(local_ms: float, local_units: float, group=None):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason sampling during the timed region.
+    Only samples stamped between entering and leaving the `with` block count
+    (nvidia-smi needs a moment to start, so it is started 0.3 s earlier)."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    STAMP = "%Y/%m/%d %H:%M:%S.%f"
 
     def __init__(self, index: int, interval_ms: int = 100):
         self.index = index
         self.interval_ms = interval_ms
         self.proc = None
+        self.t0 = self.t1 = None
+        self.out = ""
 
     def __enter__(self):
         try:
@@ -111,10 +182,11 @@ class ClockSampler:
         except OSError:
             self.proc = None
         time.sleep(0.3)
+        self.t0 = datetime.datetime.now()
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
+        self.t1 = datetime.datetime.now()
         if self.proc is not None:
             time.sleep(0.15)
             self.proc.terminate()
@@ -125,18 +197,39 @@ class ClockSampler:
                 self.out, _ = self.proc.communicate()
 
     def summary(self):
-        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
-        loaded = [s for s in sm if mx and s >= 0.3 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()),
-                                   default=None)}
+        return summarize_clocks(self.out or "", self.t0, self.t1, self.STAMP)
+
+
+def summarize_clocks(text, t0=None, t1=None, stamp="%Y/%m/%d %H:%M:%S.%f"):
+    """Median SM clock (samples above 0.3 of the maximum), maximum, the
+    throttle reasons seen and the peak power, over the rows of nvidia-smi
+    output stamped inside [t0, t1] (all rows when none is)."""
+    rows = [r for r in csv.reader(io.StringIO(text)) if len(r) >= 10]
+
+    def stamped(r):
+        try:
+            return datetime.datetime.strptime(r[0].strip(), stamp)
+        except ValueError:
+            return None
+    if t0 is not None and t1 is not None:
+        inside = [r for r in rows if (lambda ts: ts is not None and t0 <= ts <= t1)(stamped(r))]
+        rows = inside or rows
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+    def num(v):
+        try:
+            return float(v)
+        except ValueError:
+            return None
+    sm = [x for x in (num(r[2]) for r in rows) if x is not None]
+    mx = [x for x in (num(r[3]) for r in rows) if x is not None]
+    pw = [x for x in (num(r[4]) for r in rows) if x is not None]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].strip() == "Active"})
+    loaded = [v for v in sm if mx and v >= 0.3 * max(mx)] or sm
+    return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
 
 
 def blas_threads():
@@ -238,15 +331,19 @@ def main():
     ap.add_argument("--workload", default="h4096")
     ap.add_argument("--t", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--split", type=int, default=0,
-                    help="split flags: 1 = Y from the (H, H_lo) pair, 2 = dX from the (dH, dH_lo) pair")
+    ap.add_argument("--mode", default="auto", choices=["auto", "fast", "accurate"],
+                    help="precision mode: accurate (library default: Y and dX over the bf16 pair), fast (Y and dX "
+                         "from the high half), auto (fast where its parity test meets the bar, else accurate)")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of each end-to-end leg (default: --steps, so it runs as long as the headline loop)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-t", action="store_true", help="time only the headline shard count")
     ap.add_argument("--no-recompute", action="store_true", help="skip the activation-recomputation leg")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
-    ap.add_argument("--clock-interval-ms", type=int, default=100,
+    ap.add_argument("--no-steady", action="store_true", help="skip the two-second steady-state leg")
+    ap.add_argument("--no-accurate-leg", action="store_true",
+                    help="with the fast mode timed, skip timing the accurate mode beside it")
+    ap.add_argument("--clock-interval-ms", type=int, default=50,
                     help="nvidia-smi sampling period during the timed region")
     args = ap.parse_args()
 
@@ -280,20 +377,21 @@ def main():
     Z = torch.empty(T, f, dtype=torch.float32, device="cuda")
     H, H_lo, Y, dH, dH_lo = e(T, f), e(T, f), e(T, h), e(T, f), e(T, f)
     dX, dA, dB, da, db = e(T, h), e(h, f), e(f, h), e(f), e(h)
-    split = args.split
-    H_lo2 = H_lo if split & 1 else None
-    dH_lo2 = dH_lo if split & 2 else None
+    mode_name = pick_mode(args.mode, wl.name)
+    mode = MODES[mode_name]
+    H_lo2 = None if mode & 1 else H_lo
+    dH_lo2 = None if mode & 2 else dH_lo
     ws = binding.make_workspace(T, h, f, t)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
-    def step(evs=None):
+    def step(evs=None, lo_y=H_lo2, lo_dx=dH_lo2):
         calls = (
             lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, H_lo, ws, sh),
-            lambda: binding.mlp_tp_fc2_forward(H, H_lo2, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
+            lambda: binding.mlp_tp_fc2_forward(H, lo_y, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
             lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, dH_lo, da, ws, sh),
             lambda: binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t, dB, db, ws, sh),
-            lambda: binding.mlp_tp_fc1_backward_data(dH, dH_lo2, dev["A"], T, h, f, t, dX, ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_data(dH, lo_dx, dev["A"], T, h, f, t, dX, ws, sh),
             lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t, dA, ws, sh),
         )
         for i, c in enumerate(calls):
@@ -328,17 +426,58 @@ def main():
         dist.barrier()
     binding.mlp_tp_check(ws, sh)
     local_ms = start.elapsed_time(end)
-    n_ev = max(10, args.steps // 4)
+    # per-stage times (events between the stage calls), with the clocks of
+    # this window: the roofline's peak follows them
+    n_ev = max(10, args.steps // 4, int(0.3e3 / max(local_ms / args.steps, 1e-3)) + 1)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(n_ev)]
-    for k in range(n_ev):
-        step(ev[k])
     torch.cuda.synchronize()
+    with ClockSampler(local, args.clock_interval_ms) as clk_stages:
+        for k in range(n_ev):
+            step(ev[k])
+        torch.cuda.synchronize()
     binding.mlp_tp_check(ws, sh)
     stage_ms = {s: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(n_ev))
                 for i, s in enumerate(STAGES)}
     max_ms, total_flops = reduce_max_sum(local_ms, float(wl.flops) * args.steps)
     value = total_flops / (max_ms * 1e-3) / 1e12
     ms_per_step = max_ms / args.steps
+
+    def timed_loop(n, **kw):
+        """Device time of n back-to-back steps (events around the loop only),
+        max over ranks, and the clocks sampled meanwhile."""
+        s_l, e_l = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local, args.clock_interval_ms) as c:
+            s_l.record(stream)
+            for _ in range(n):
+                step(**kw)
+            e_l.record(stream)
+            torch.cuda.synchronize()
+        binding.mlp_tp_check(ws, sh)
+        ms_l, fl_l = reduce_max_sum(s_l.elapsed_time(e_l), float(wl.flops) * n)
+        return ms_l, fl_l, c.summary()
+
+    # ------------------------------------------------ the accurate (default) mode beside the fast one
+    accurate = None
+    if mode != MODES["accurate"] and not args.no_accurate_leg:
+        for _ in range(3):
+            step(lo_y=H_lo, lo_dx=dH_lo)
+        ms_a, fl_a, clk_a = timed_loop(args.steps, lo_y=H_lo, lo_dx=dH_lo)
+        accurate = {"value": fl_a / (ms_a * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_a / args.steps,
+                    "steps": args.steps, "clocks": clk_a,
+                    "api": "the same stage calls with the low half of the pair in the Y and dX GEMMs "
+                           "(the library's default mode)"}
+
+    # ------------------------------------------------ steady state: the same loop for >= 2 s
+    steady = None
+    if not args.no_steady:
+        n_s = max(args.steps, int(STEADY_SECONDS * 1e3 / max(ms_per_step, 1e-3)) + 1)
+        ms_s, fl_s, clk_s = timed_loop(n_s)
+        steady = {"value": fl_s / (ms_s * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_s / n_s, "steps": n_s,
+                  "seconds": ms_s * 1e-3, "clocks": clk_s,
+                  "ms_x_mhz": (ms_s / n_s) * clk_s["sm_mhz"] if clk_s.get("sm_mhz") else None}
 
     # ------------------------------------------------ the workload's other shard counts
     # Same device-resident step (stage calls) for every other t the workload
@@ -425,9 +564,9 @@ def main():
         ws_r = binding.make_recompute_workspace(T, h, f, t)
 
         def step_r():
-            binding.mlp_tp_forward_recompute(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, split,
+            binding.mlp_tp_forward_recompute(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, mode,
                                              Y, ws_r, sh)
-            binding.mlp_tp_backward_recompute(dev["dY"], dev["X"], dev["A"], dev["a"], dev["B"], T, h, f, t, split,
+            binding.mlp_tp_backward_recompute(dev["dY"], dev["X"], dev["A"], dev["a"], dev["B"], T, h, f, t, mode,
                                               dX, dA, da, dB, db, ws_r, sh)
 
         for _ in range(3):
@@ -488,9 +627,9 @@ def main():
             if k >= 2:
                 s_cmp.wait_event(out_done[k - 2])  # step k-2's outputs in set k % 2 copied out
             cs = s_cmp.cuda_stream
-            binding.mlp_tp_forward(d_in["X"], d_in["A"], d_in["a"], d_in["B"], d_in["b"], T, h, f, t, split,
+            binding.mlp_tp_forward(d_in["X"], d_in["A"], d_in["a"], d_in["B"], d_in["b"], T, h, f, t, mode,
                                    d_out["Y"], Z, H, H_lo, ws, cs)
-            binding.mlp_tp_backward(d_in["dY"], d_in["X"], d_in["A"], d_in["B"], Z, H, H_lo, T, h, f, t, split,
+            binding.mlp_tp_backward(d_in["dY"], d_in["X"], d_in["A"], d_in["B"], Z, H, H_lo, T, h, f, t, mode,
                                     d_out["dX"], d_out["dA"], d_out["da"], d_out["dB"], d_out["db"], ws, cs)
             c_done.record(s_cmp)
             cmp_done.append(c_done)
@@ -540,36 +679,19 @@ def main():
 
     # ------------------------------------------------ roofline of the dominant kernel
     peaks, peak_src = load_peaks()
-    dom = max(STAGES, key=lambda s: stage_ms[s])
-    products = dict(STAGE_PRODUCTS)
-    products["fc2_forward"] += 1 if split & 1 else 0
-    products["fc1_backward_data"] += 1 if split & 2 else 0
-    gemm_flops = 2.0 * T * h * f * products[dom]
-    achieved = gemm_flops / (stage_ms[dom] * 1e-3) / 1e12
-    # Peak for the roofline: the measured sustained bf16 figure (cuBLAS looped
-    # for seconds under the power cap) when the clocks sampled in the timed
-    # region show the power cap or a clock well below its maximum, the burst
-    # figure otherwise.  Both fractions are reported.
+    roofline = roofline_entry(stage_ms, mode, T, h, f, clk_stages.summary(), peaks, peak_src)
+    roofline["traffic"] = traffic_for(roofline["stage"], wl, t)
+    products = stage_products(mode)
     clocks = clk.summary()
-    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    capped = "sw_power_cap" in clocks.get("reasons", []) or (
-        clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"])
-    peak = peak_sustained if capped else peak_burst
-    peak_kind = "bf16_tflops_sustained (power cap seen in the timed region)" if capped else "bf16_tflops (burst)"
-    roofline = {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved,
-                "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                "peak_source": f"{peak_src} {peak_kind}",
-                "frac_of_burst": achieved / peak_burst, "frac_of_sustained": achieved / peak_sustained,
-                "traffic": traffic_for(dom, wl, t),
-                "algorithmic_flops_per_launch": gemm_flops, "avg_launch_ms": stage_ms[dom]}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, bf16)",
-        "config": dict(workload_config(wl, t, world), precision=precision_note(split),
+        "config": dict(workload_config(wl, t, world), precision=precision_note(mode),
                        tensor_flops_per_step=2.0 * T * h * f * sum(products.values())),
+        "precision_mode": precision_mode_note(mode_name, args.mode, wl.name),
         "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_DENSE_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * value / world / float(peaks.get("bf16_tflops", 1713.1)),
         # cuBLAS looped for seconds under the power cap, like this 200-step region
@@ -584,7 +706,12 @@ def main():
                 "resident_parameters": e2e_resident},
         "gpu_launches": launches,
         "clocks": clocks,
+        "ms_x_mhz": ms_per_step * clocks["sm_mhz"] if clocks.get("sm_mhz") else None,
     }
+    if accurate is not None:
+        line["accurate"] = accurate
+    if steady is not None:
+        line["steady"] = steady
     if graph is not None:
         line["graph"] = graph
     if recompute is not None:
@@ -595,11 +722,22 @@ def main():
     return 0
 
 
-def precision_note(split):
-    y = "(H, H_lo) pair" if split & 1 else "bf16 H"
-    dx = "(dH, dH_lo) pair" if split & 2 else "bf16 dH"
+def precision_note(mode):
+    y = "bf16 H (high half)" if mode & 1 else "(H, H_lo) pair"
+    dx = "bf16 dH (high half)" if mode & 2 else "(dH, dH_lo) pair"
     return (f"bf16 inputs, fp32 accumulation; Z saved fp32; Y from {y}; dX from {dx}; dA, dB from the "
             f"(hi, lo) bf16 pairs; da from fp32 dH")
+
+
+def precision_mode_note(mode_name, requested, wl_name):
+    if mode_name == "fast":
+        why = (f"fast mode: Y and dX from the high half of the bf16 activation pair; its GPU parity test on "
+               f"the {wl_name} workload meets the 1e-2·(|oracle|+1) bar"
+               + (" (chosen by --mode auto)" if requested == "auto" else "")
+               + "; the library's default (accurate) mode is timed in `accurate`")
+    else:
+        why = "accurate mode (the library's default): Y and dX over both halves of the bf16 activation pair"
+    return {"timed": mode_name, "note": why}
 
 
 def traffic_for(stage, wl, t):

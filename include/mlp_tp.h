@@ -32,11 +32,12 @@
  *    The backward forms dH = (dY·Bᵀ) ⊙ g'(Z) in fp32 and keeps it as the
  *    same kind of pair.  The weight gradients dA = Xᵀ·dH and dB = Hᵀ·dY
  *    always use both halves of the pair (two bf16 tensor-core products);
- *    Y and dX use only the high half unless the split flags below ask for
- *    both.  da is summed from the fp32 dH before rounding.  With bf16-rounded
- *    intermediates alone, the gradients of a unit-scale batch of a few
- *    thousand tokens already differ from the exact block by more than
- *    1e-2·(|exact| + 1); the pairs keep them well inside it.
+ *    Y and dX use both halves in the default mode (MLP_TP_ACCURATE) and the
+ *    high half only in the fast modes below.  da is summed from the fp32 dH
+ *    before rounding.  With bf16-rounded intermediates alone, the gradients
+ *    of a unit-scale batch of a few thousand tokens already differ from the
+ *    exact block by more than 1e-2·(|exact| + 1); the pairs keep them well
+ *    inside it.
  *  - Every device pointer must be 16-byte aligned.  Inputs are only read;
  *    outputs are overwritten (never accumulated into).  Outputs must not
  *    alias inputs or each other.
@@ -94,23 +95,38 @@ typedef enum {
  * than the GPU has CTA pairs).  Returns 0 for an invalid shape. */
 size_t mlp_tp_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
 
-/* Split flags of the composite calls: which second-layer products also use
- * the low half of the activation pair.  The weight gradients always do. */
+/* Precision mode of the composite calls: which second-layer products also
+ * use the low half of the activation pair.  The weight gradients always do.
+ *
+ * 0 (MLP_TP_ACCURATE) is the default: Y = Σ_i (H_i + H_lo_i)·B_i + b and
+ * dX = Σ_i (dH_i + dH_lo_i)·A_iᵀ, which meets
+ * max|result − exact| <= 1e-2·(|exact| + 1) on every workload the tests run.
+ *
+ * The fast flags drop the low half from one or both of those products (half
+ * their tensor-core work).  The error they add grows like
+ * 2^-9·sqrt(f)·rms(B)·rms(H) for Y (and the same with A, dH for dX), so it
+ * depends on the data, not on the shape alone.  Known cases:
+ *   - meets the bar: the tiny (T=64, h=256, f=1024), GPT-2-medium (T=8192,
+ *     h=1024, f=4096), h=4096 (T=4096, h=4096, f=16384, weights
+ *     ~N(0, 0.0025)) and 175B-class (T=8192, h=12288, f=49152, weights
+ *     ~N(0, 0.006)) workloads;
+ *   - exceeds it: the 8.3B-class workload (T=16384, h=3072, f=12288,
+ *     weights ~N(0, 0.02)), Y by 1.08x and dX by 1.14x of the tolerance. */
 typedef enum {
-  MLP_TP_SPLIT_NONE = 0,
-  MLP_TP_SPLIT_FC2_FORWARD = 1,       /* Y  = Σ_i (H_i + H_lo_i)·B_i + b    */
-  MLP_TP_SPLIT_FC1_BACKWARD_DATA = 2, /* dX = Σ_i (dH_i + dH_lo_i)·A_iᵀ     */
-  MLP_TP_SPLIT_ALL = 3
-} mlp_tp_split_t;
+  MLP_TP_ACCURATE = 0,
+  MLP_TP_FAST_FC2_FORWARD = 1,       /* Y  = Σ_i H_i·B_i + b       (high half only) */
+  MLP_TP_FAST_FC1_BACKWARD_DATA = 2, /* dX = Σ_i dH_i·A_iᵀ         (high half only) */
+  MLP_TP_FAST = 3                    /* both */
+} mlp_tp_mode_t;
 
 /* ---------------------------------------------------------------- forward */
 
 /* Whole forward: mlp_tp_fc1_forward then mlp_tp_fc2_forward (the latter
- * given H_lo when `split` has MLP_TP_SPLIT_FC2_FORWARD).  Writes Y[T,h] and
+ * given H_lo unless `mode` has MLP_TP_FAST_FC2_FORWARD).  Writes Y[T,h] and
  * saves Z[T,f] (fp32), H[T,f] and H_lo[T,f] for the backward. */
 mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a,
                             const void* B, const void* b,
-                            int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                            int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
                             void* Y, void* Z, void* H, void* H_lo,
                             void* ws, size_t ws_bytes, void* stream);
 
@@ -136,12 +152,12 @@ mlp_status_t mlp_tp_fc2_forward(const void* H, const void* H_lo, const void* B, 
 
 /* Whole backward, given dY and Z, H, H_lo saved by the forward:
  * mlp_tp_fc2_backward_data (dH pair into the workspace),
- * mlp_tp_fc2_backward_weight, mlp_tp_fc1_backward_data (given dH_lo when
- * `split` has MLP_TP_SPLIT_FC1_BACKWARD_DATA) and mlp_tp_fc1_backward_weight.
+ * mlp_tp_fc2_backward_weight, mlp_tp_fc1_backward_data (given dH_lo unless
+ * `mode` has MLP_TP_FAST_FC1_BACKWARD_DATA) and mlp_tp_fc1_backward_weight.
  * `da` and `db` may be NULL (bias gradients not wanted). */
 mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A,
                              const void* B, const void* Z, const void* H, const void* H_lo,
-                             int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                             int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
                              void* dX, void* dA, void* da, void* dB, void* db,
                              void* ws, size_t ws_bytes, void* stream);
 
@@ -190,18 +206,18 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
  * backward of mlp_tp_backward.  Both need
  * mlp_tp_recompute_workspace_bytes(T, h, f, t) bytes of workspace (the
  * ordinary workspace plus T·f·8 bytes for Z, H, H_lo).  Same conventions
- * and split flags as mlp_tp_forward / mlp_tp_backward. */
+ * and modes as mlp_tp_forward / mlp_tp_backward. */
 size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
 
 mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* a,
                                       const void* B, const void* b,
-                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
                                       void* Y,
                                       void* ws, size_t ws_bytes, void* stream);
 
 mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void* A,
                                        const void* a, const void* B,
-                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t split,
+                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
                                        void* dX, void* dA, void* da, void* dB, void* db,
                                        void* ws, size_t ws_bytes, void* stream);
 
@@ -226,17 +242,21 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
  * work overlaps on the GPU (different streams, or several host threads
  * without ordering) race on it; calls ordered on one stream do not.  No
  * call allocates or frees memory.  Same pointer, alignment and device rules
- * as the other entry points; dY may be NULL when T == 0 (db is zero-filled). */
+ * as the other entry points; dY may be NULL when T == 0 (db is zero-filled).
+ * The path keeps its own device status word beside the array;
+ * mlp_tp_check(NULL, stream) reads it. */
 mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, int64_t h, void* db, void* stream);
 
 /* ------------------------------------------------------------ diagnostics */
 
 /* Synchronises `stream`, then reads and clears the device status word in
- * `ws`.  Returns MLP_OK, MLP_ERR_TIMEOUT (a kernel's bounded wait ran out;
- * its outputs are undefined, the CUDA context stays usable), MLP_ERR_BOUNDS
- * (only from a library built with -DMLPTP_BOUNDS_CHECK: a plain global
- * access outside its buffer was found and skipped) or MLP_ERR_CUDA (the
- * stream reported an error). */
+ * `ws` (ws == NULL: the status word of mlp_tp_fc2_bias_grad_noalloc on the
+ * current device).  Returns MLP_OK, MLP_ERR_TIMEOUT (a kernel's bounded wait
+ * ran out; that launch's outputs, and anything later on the context, are not
+ * to be trusted: a copy the kernel could not wait for may still have landed
+ * after it returned), MLP_ERR_BOUNDS (only from a library built with
+ * -DMLPTP_BOUNDS_CHECK: a plain global access outside its buffer was found
+ * and skipped) or MLP_ERR_CUDA (the stream reported an error). */
 mlp_status_t mlp_tp_check(void* ws, void* stream);
 
 /* Static, NUL-terminated name of a status code. */

@@ -56,11 +56,11 @@ _SIGS = {
     "mlp_tp_set_debug_flags": ([ctypes.c_uint32], None),
 }
 
-# split flags of the composite calls (mlp_tp_split_t)
-SPLIT_NONE = 0
-SPLIT_FC2_FORWARD = 1
-SPLIT_FC1_BACKWARD_DATA = 2
-SPLIT_ALL = 3
+# precision modes of the composite calls (mlp_tp_mode_t); 0 is the accurate default
+ACCURATE = 0
+FAST_FC2_FORWARD = 1
+FAST_FC1_BACKWARD_DATA = 2
+FAST = 3
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -149,10 +149,10 @@ def make_workspace(T: int, h: int, f: int, t: int, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def mlp_tp_forward(X, A, a, B, b, T, h, f, t, split, Y, Z, H, H_lo, ws, stream=None):
+def mlp_tp_forward(X, A, a, B, b, T, h, f, t, mode, Y, Z, H, H_lo, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"), _addr(b, "b"),
-                                T, h, f, t, split, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"),
+                                T, h, f, t, mode, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"),
                                 _addr(H_lo, "H_lo"), w, wn, _stream(stream)))
 
 
@@ -168,10 +168,10 @@ def mlp_tp_fc2_forward(H, H_lo, B, b, T, h, f, t, Y, ws, stream=None):
                                     T, h, f, t, _addr(Y, "Y"), w, wn, _stream(stream)))
 
 
-def mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, split, dX, dA, da, dB, db, ws, stream=None):
+def mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, mode, dX, dA, da, dB, db, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_backward(_addr(dY, "dY"), _addr(X, "X"), _addr(A, "A"), _addr(B, "B"), _addr(Z, "Z"),
-                                 _addr(H, "H"), _addr(H_lo, "H_lo"), T, h, f, t, split, _addr(dX, "dX"),
+                                 _addr(H, "H"), _addr(H_lo, "H_lo"), T, h, f, t, mode, _addr(dX, "dX"),
                                  _addr(dA, "dA"), _addr(da, "da", True), _addr(dB, "dB"), _addr(db, "db", True),
                                  w, wn, _stream(stream)))
 
@@ -213,17 +213,17 @@ def make_recompute_workspace(T: int, h: int, f: int, t: int, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def mlp_tp_forward_recompute(X, A, a, B, b, T, h, f, t, split, Y, ws, stream=None):
+def mlp_tp_forward_recompute(X, A, a, B, b, T, h, f, t, mode, Y, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_forward_recompute(_addr(X, "X", T == 0), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"),
-                                          _addr(b, "b"), T, h, f, t, split, _addr(Y, "Y", T == 0), w, wn,
+                                          _addr(b, "b"), T, h, f, t, mode, _addr(Y, "Y", T == 0), w, wn,
                                           _stream(stream)))
 
 
-def mlp_tp_backward_recompute(dY, X, A, a, B, T, h, f, t, split, dX, dA, da, dB, db, ws, stream=None):
+def mlp_tp_backward_recompute(dY, X, A, a, B, T, h, f, t, mode, dX, dA, da, dB, db, ws, stream=None):
     w, wn = _ws(ws)
     _check(lib().mlp_tp_backward_recompute(_addr(dY, "dY", T == 0), _addr(X, "X", T == 0), _addr(A, "A"),
-                                           _addr(a, "a"), _addr(B, "B"), T, h, f, t, split,
+                                           _addr(a, "a"), _addr(B, "B"), T, h, f, t, mode,
                                            _addr(dX, "dX", T == 0), _addr(dA, "dA"), _addr(da, "da", True),
                                            _addr(dB, "dB"), _addr(db, "db", True), w, wn, _stream(stream)))
 
@@ -234,7 +234,9 @@ def mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db, stream=None):
 
 
 def mlp_tp_check(ws, stream=None):
-    w, _ = _ws(ws)
+    """Sync the stream and read the workspace's status word (ws=None: the
+    allocation-free entry point's own status word)."""
+    w = None if ws is None else _ws(ws)[0]
     _check(lib().mlp_tp_check(w, _stream(stream)))
 
 

@@ -21,26 +21,27 @@ def alloc_outputs(T: int, h: int, f: int, device="cuda", with_bias_grads: bool =
 
 
 def forward(inp: Dict[str, torch.Tensor], t: int, out: Dict[str, torch.Tensor], ws: torch.Tensor,
-            split: int = binding.SPLIT_NONE, stream=None) -> None:
+            mode: int = binding.ACCURATE, stream=None) -> None:
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
-    binding.mlp_tp_forward(inp["X"], inp["A"], inp["a"], inp["B"], inp["b"], T, h, f, t, split,
+    binding.mlp_tp_forward(inp["X"], inp["A"], inp["a"], inp["B"], inp["b"], T, h, f, t, mode,
                            out["Y"], out["Z"], out["H"], out["H_lo"], ws, stream)
 
 
 def backward(inp: Dict[str, torch.Tensor], t: int, out: Dict[str, torch.Tensor], ws: torch.Tensor,
-             split: int = binding.SPLIT_NONE, stream=None) -> None:
+             mode: int = binding.ACCURATE, stream=None) -> None:
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
     binding.mlp_tp_backward(inp["dY"], inp["X"], inp["A"], inp["B"], out["Z"], out["H"], out["H_lo"],
-                            T, h, f, t, split, out["dX"], out["dA"], out.get("da"), out["dB"], out.get("db"),
+                            T, h, f, t, mode, out["dX"], out["dA"], out.get("da"), out["dB"], out.get("db"),
                             ws, stream)
 
 
 def forward_backward(inp: Dict[str, torch.Tensor], t: int, out: Optional[Dict[str, torch.Tensor]] = None,
-                     ws: Optional[torch.Tensor] = None, split: int = binding.SPLIT_NONE,
+                     ws: Optional[torch.Tensor] = None, mode: int = binding.ACCURATE,
                      check: bool = True) -> Dict[str, torch.Tensor]:
-    """Run forward then backward on the current stream; returns the outputs."""
+    """Run forward then backward on the current stream; returns the outputs.
+    ``mode`` is the precision mode (binding.ACCURATE by default)."""
     T, h = inp["X"].shape
     f = inp["A"].shape[1]
     dev = inp["X"].device
@@ -48,8 +49,8 @@ def forward_backward(inp: Dict[str, torch.Tensor], t: int, out: Optional[Dict[st
         out = alloc_outputs(T, h, f, dev)
     if ws is None:
         ws = binding.make_workspace(T, h, f, t, dev)
-    forward(inp, t, out, ws, split)
-    backward(inp, t, out, ws, split)
+    forward(inp, t, out, ws, mode)
+    backward(inp, t, out, ws, mode)
     if check:
         binding.mlp_tp_check(ws)
     return out

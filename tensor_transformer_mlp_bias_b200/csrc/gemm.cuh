@@ -134,10 +134,8 @@ constexpr unsigned int STATUS_BOUNDS = 8u;
 __device__ __forceinline__ bool index_ok(long long last, long long n, unsigned int* status, unsigned int site) {
 #ifdef MLPTP_BOUNDS_CHECK
   if (last < 0 || last >= n) {
-    if (status != nullptr) {  // the allocation-free path has no status word
-      atomicCAS(status, 0u, STATUS_BOUNDS);
-      atomicCAS(status + 1, 0u, site);
-    }
+    atomicCAS(status, 0u, STATUS_BOUNDS);
+    atomicCAS(status + 1, 0u, site);
     return false;
   }
 #else
@@ -555,8 +553,12 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
       // exit: the barrier owner waits for the last arming of every stage
       // (immediate when the tensor-core warp already consumed it).  In pair
       // mode the leader's barriers also count the peer's copies.
+      // A drain that runs out is recorded like any other timeout: the copy may
+      // still land after the CTA has exited, so nothing the grid produced (nor
+      // anything later on this context) can be trusted.
       for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s)) mbar_drain(&ctl->full[s], (issued_phase >> s) & 1u, budget);
+        if ((issued_mask & (1u << s)) && !mbar_drain(&ctl->full[s], (issued_phase >> s) & 1u, budget))
+          record_timeout(p, abort_flag, 0x600u | static_cast<unsigned int>(s));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
       } else {
         mma_commit(&ctl->mma_done);
       }
-      mbar_drain(&ctl->mma_done, 0u, budget);
+      if (!mbar_drain(&ctl->mma_done, 0u, budget)) record_timeout(p, abort_flag, 0x700u);
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -555,6 +555,25 @@ float* tail_scratch(void* ws, const Shape& s) {
   return reinterpret_cast<float*>(static_cast<char*>(ws) + tail_offset(s));
 }
 
+// Synchronises the stream, then reads and clears a device status word pair
+// (code, site).
+mlp_status_t read_status_word(unsigned int* status, cudaStream_t cs) {
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word[2] = {0u, 0u};
+  e = cudaMemcpy(word, status, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (word[0] == 0u) return MLP_OK;
+  const unsigned int zero[2] = {0u, 0u};
+  e = cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  if (word[0] == STATUS_TIMEOUT)
+    return fail(MLP_ERR_TIMEOUT, "a kernel wait ran out of its budget (site 0x%x)", word[1]);
+  if (word[0] == STATUS_BOUNDS)
+    return fail(MLP_ERR_BOUNDS, "an index fell outside its buffer (site 0x%x; bounds-checking build)", word[1]);
+  return fail(MLP_ERR_CUDA, "device status word holds unknown code %u", word[0]);
+}
+
 // ---------------------------------------------------------------- stages
 mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H, void* H_lo,
                          void* ws, const Launch& L) {
@@ -665,10 +684,19 @@ mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws,
   return current_device(L.dev, L.sms);
 }
 
-mlp_status_t check_split(int32_t split) {
-  if (split < 0 || split > MLP_TP_SPLIT_ALL) return fail(MLP_ERR_INVALID_ARG, "split flags %d out of range", split);
+mlp_status_t check_mode(int32_t mode) {
+  if (mode < MLP_TP_ACCURATE || mode > MLP_TP_FAST) return fail(MLP_ERR_INVALID_ARG, "precision mode %d out of range", mode);
   return MLP_OK;
 }
+
+// The low half of the pair feeds Y (and dX) unless the mode asks for the fast form.
+const void* fc2_lo(int32_t mode, const void* H_lo) { return (mode & MLP_TP_FAST_FC2_FORWARD) ? nullptr : H_lo; }
+const void* fc1_bwd_lo(int32_t mode, const void* dH_lo) {
+  return (mode & MLP_TP_FAST_FC1_BACKWARD_DATA) ? nullptr : dH_lo;
+}
+
+// Status word of the allocation-free entry point (defined with it below).
+mlp_status_t noalloc_check(cudaStream_t cs);
 
 }  // namespace
 
@@ -706,11 +734,11 @@ mlp_status_t mlp_tp_fc2_forward(const void* H, const void* H_lo, const void* B, 
 }
 
 mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a, const void* B, const void* b, int64_t T,
-                            int64_t h, int64_t f, int32_t t, int32_t split, void* Y, void* Z, void* H, void* H_lo,
+                            int64_t h, int64_t f, int32_t t, int32_t mode, void* Y, void* Z, void* H, void* H_lo,
                             void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
   Launch L;
-  mlp_status_t st = check_split(split);
+  mlp_status_t st = check_mode(mode);
   if (st != MLP_OK) return st;
   st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
                     {Y, "Y", false, s.T == 0}, {Z, "Z", false, s.T == 0}, {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}},
@@ -718,7 +746,7 @@ mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a, const v
   if (st != MLP_OK) return st;
   st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L);
   if (st != MLP_OK) return st;
-  return fc2_forward(s, H, (split & MLP_TP_SPLIT_FC2_FORWARD) ? H_lo : nullptr, B, b, Y, ws, L);
+  return fc2_forward(s, H, fc2_lo(mode, H_lo), B, b, Y, ws, L);
 }
 
 mlp_status_t mlp_tp_fc2_backward_data(const void* dY, const void* B, const void* Z, int64_t T, int64_t h, int64_t f,
@@ -766,11 +794,11 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
 }
 
 mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const void* B, const void* Z, const void* H,
-                             const void* H_lo, int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* dX,
+                             const void* H_lo, int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode, void* dX,
                              void* dA, void* da, void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
   Launch L;
-  mlp_status_t st = check_split(split);
+  mlp_status_t st = check_mode(mode);
   if (st != MLP_OK) return st;
   st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {B, "B", false}, {Z, "Z", false, s.T == 0},
                     {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
@@ -781,9 +809,7 @@ mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const
   void* dH_lo = static_cast<char*>(ws) + dh_lo_offset(s);
   if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
-  if ((st = fc1_backward_data(s, dH, (split & MLP_TP_SPLIT_FC1_BACKWARD_DATA) ? dH_lo : nullptr, A, dX, ws, L)) !=
-      MLP_OK)
-    return st;
+  if ((st = fc1_backward_data(s, dH, fc1_bwd_lo(mode, dH_lo), A, dX, ws, L)) != MLP_OK) return st;
   return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
 }
 
@@ -796,11 +822,11 @@ size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t
 }
 
 mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* a, const void* B, const void* b,
-                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* Y, void* ws,
+                                      int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode, void* Y, void* ws,
                                       size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
   Launch L;
-  mlp_status_t st = check_split(split);
+  mlp_status_t st = check_mode(mode);
   if (st != MLP_OK) return st;
   st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
                     {Y, "Y", false, s.T == 0}},
@@ -811,15 +837,15 @@ mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* 
   void* H = w + recompute_h_offset(s);
   void* H_lo = w + recompute_hlo_offset(s);
   if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
-  return fc2_forward(s, H, (split & MLP_TP_SPLIT_FC2_FORWARD) ? H_lo : nullptr, B, b, Y, ws, L);
+  return fc2_forward(s, H, fc2_lo(mode, H_lo), B, b, Y, ws, L);
 }
 
 mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void* A, const void* a, const void* B,
-                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t split, void* dX, void* dA,
+                                       int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode, void* dX, void* dA,
                                        void* da, void* dB, void* db, void* ws, size_t ws_bytes, void* stream) {
   Shape s{T, h, f, t};
   Launch L;
-  mlp_status_t st = check_split(split);
+  mlp_status_t st = check_mode(mode);
   if (st != MLP_OK) return st;
   st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false},
                     {B, "B", false}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
@@ -836,29 +862,14 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
   if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
-  if ((st = fc1_backward_data(s, dH, (split & MLP_TP_SPLIT_FC1_BACKWARD_DATA) ? dH_lo : nullptr, A, dX, ws, L)) !=
-      MLP_OK)
-    return st;
+  if ((st = fc1_backward_data(s, dH, fc1_bwd_lo(mode, dH_lo), A, dX, ws, L)) != MLP_OK) return st;
   return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
 }
 
 mlp_status_t mlp_tp_check(void* ws, void* stream) {
-  if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaStreamSynchronize(cs);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  unsigned int word[2] = {0u, 0u};
-  e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status word");
-  if (word[0] == 0u) return MLP_OK;
-  const unsigned int zero[2] = {0u, 0u};
-  e = cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace status word");
-  if (word[0] == STATUS_TIMEOUT)
-    return fail(MLP_ERR_TIMEOUT, "a kernel wait ran out of its budget (site 0x%x)", word[1]);
-  if (word[0] == STATUS_BOUNDS)
-    return fail(MLP_ERR_BOUNDS, "an index fell outside its buffer (site 0x%x; bounds-checking build)", word[1]);
-  return fail(MLP_ERR_CUDA, "device status word holds unknown code %u", word[0]);
+  if (ws == nullptr) return noalloc_check(cs);
+  return read_status_word(static_cast<unsigned int*>(ws), cs);
 }
 
 const char* mlp_tp_status_string(mlp_status_t status) {
@@ -894,23 +905,39 @@ void mlp_tp_set_debug_flags(uint32_t flags) { g_debug_flags.store(flags); }
 namespace {
 
 constexpr size_t NOALLOC_MAX_PARTIALS = size_t(1) << 20;  // 4 MiB of fp32
+constexpr int NOALLOC_MAX_DEVICES = 64;
 static __device__ __align__(256) float g_noalloc_partials[NOALLOC_MAX_PARTIALS];
+// The path's own status word (code, site), the counterpart of the one a
+// workspace holds: the bounds-checking build records out-of-range indices
+// here; mlp_tp_check(NULL, stream) reads and clears it.
+static __device__ __align__(16) unsigned int g_noalloc_status[2];
 
-// Host code may not use g_noalloc_partials directly (on the host it only
-// names a stand-in); its device address is looked up once per device, with
-// that device current.
-float* g_noalloc_ptr[64] = {};
+// Host code may not use these arrays directly (on the host their names only
+// stand for host-side placeholders); their device addresses are looked up
+// once per device, with that device current.
+struct NoallocScratch {
+  float* partials = nullptr;
+  unsigned int* status = nullptr;
+};
+NoallocScratch g_noalloc[NOALLOC_MAX_DEVICES];
 std::mutex g_noalloc_mu;
 
-mlp_status_t noalloc_scratch(int dev, float** out) {
+mlp_status_t noalloc_scratch(int dev, NoallocScratch* out) {
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES)
+    return fail(MLP_ERR_UNSUPPORTED_DEVICE, "device ordinal %d out of range for the static scratch", dev);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocScratch& d = g_noalloc[dev];
+  if (d.partials == nullptr) {
     void* p = nullptr;
+    void* q = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static column-sum scratch)");
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
+    e = cudaGetSymbolAddress(&q, g_noalloc_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static status word)");
+    d.status = static_cast<unsigned int*>(q);
+    d.partials = static_cast<float*>(p);
   }
-  *out = g_noalloc_ptr[dev];
+  *out = d;
   return MLP_OK;
 }
 
@@ -930,9 +957,24 @@ extern "C" mlp_status_t mlp_tp_fc2_bias_grad_noalloc(const void* dY, int64_t T, 
   if (st != MLP_OK) return st;
   int dev = 0, sms = 0;
   if ((st = current_device(dev, sms)) != MLP_OK) return st;
-  float* scratch = nullptr;
+  NoallocScratch scratch;
   if ((st = noalloc_scratch(dev, &scratch)) != MLP_OK) return st;
   // Pass 1 overwrites every partial it reads back in pass 2, so nothing left
   // in the array by an earlier call is ever used.
-  return launch_colsum(dY, T, h, db, scratch, static_cast<cudaStream_t>(stream), NOALLOC_MAX_PARTIALS, nullptr);
+  return launch_colsum(dY, T, h, db, scratch.partials, static_cast<cudaStream_t>(stream), NOALLOC_MAX_PARTIALS,
+                       scratch.status);
 }
+
+namespace {
+
+// mlp_tp_check(NULL, stream): the allocation-free path's status word.
+mlp_status_t noalloc_check(cudaStream_t cs) {
+  int dev = 0, sms = 0;
+  mlp_status_t st = current_device(dev, sms);
+  if (st != MLP_OK) return st;
+  NoallocScratch scratch;
+  if ((st = noalloc_scratch(dev, &scratch)) != MLP_OK) return st;
+  return read_status_word(scratch.status, cs);
+}
+
+}  // namespace

@@ -83,7 +83,7 @@ def _reduce_scatter_tokens(x: torch.Tensor, group, async_op: bool = False):
 
 
 def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Tensor, b: torch.Tensor, *,
-            group=None, sequence_parallel: bool = False, split: int = binding.SPLIT_NONE,
+            group=None, sequence_parallel: bool = False, mode: int = binding.ACCURATE,
             ops=binding) -> Tuple[torch.Tensor, Saved]:
     """Y (full, or this rank's token rows in the sequence-parallel form) and
     the activations the backward needs.  X is the full batch, or this rank's
@@ -102,7 +102,7 @@ def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Te
     H_lo = torch.empty(T, fs, dtype=dt, device=dev)
     ops.mlp_tp_fc1_forward(X, A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws)
     P = torch.empty(T, h, dtype=dt, device=dev)
-    ops.mlp_tp_fc2_forward(H, H_lo if split & binding.SPLIT_FC2_FORWARD else None, B_i, b if rank == 0 else None,
+    ops.mlp_tp_fc2_forward(H, None if mode & binding.FAST_FC2_FORWARD else H_lo, B_i, b if rank == 0 else None,
                            T, h, fs, 1, P, ws)
     if sequence_parallel:
         Y, _ = _reduce_scatter_tokens(P, group)
@@ -113,7 +113,7 @@ def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Te
 
 
 def backward(dY: torch.Tensor, saved: Saved, A_i: torch.Tensor, B_i: torch.Tensor, *, group=None,
-             sequence_parallel: bool = False, split: int = binding.SPLIT_NONE,
+             sequence_parallel: bool = False, mode: int = binding.ACCURATE,
              ops=binding) -> Dict[str, torch.Tensor]:
     """dX (full, or this rank's token rows in the sequence-parallel form), this
     rank's shard of dA, da and dB, and db.  dY is the full gradient, or this
@@ -130,7 +130,7 @@ def backward(dY: torch.Tensor, saved: Saved, A_i: torch.Tensor, B_i: torch.Tenso
     dB, db = e(fs, h), e(h)
     ops.mlp_tp_fc2_backward_weight(saved.H, saved.H_lo, dY, T, h, fs, 1, dB, db, saved.ws)
     Q = e(T, h)
-    ops.mlp_tp_fc1_backward_data(dH, dH_lo if split & binding.SPLIT_FC1_BACKWARD_DATA else None, A_i, T, h, fs, 1,
+    ops.mlp_tp_fc1_backward_data(dH, None if mode & binding.FAST_FC1_BACKWARD_DATA else dH_lo, A_i, T, h, fs, 1,
                                  Q, saved.ws)
     # the dX reduction runs while this rank computes its dA shard
     if sequence_parallel:

@@ -113,10 +113,19 @@ def test_binding_refuses_cpu_tensors(lib):
         binding.mlp_tp_fc1_forward(x, x, x, 64, 256, 1024, 2, x, x, x, (FAKE, 1 << 30), stream=0)
 
 
-def test_split_flags_are_validated(lib):
-    st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, 1024, 2, 7, FAKE, FAKE, FAKE, FAKE,
-                            FAKE * 2, 1 << 30, None)
-    assert st == 1 and "split" in binding.mlp_tp_last_error()
+def test_precision_mode_is_validated(lib):
+    for bad in (4, 7, -1):
+        st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, 1024, 2, bad, FAKE, FAKE, FAKE, FAKE,
+                                FAKE * 2, 1 << 30, None)
+        assert st == 1 and "precision mode" in binding.mlp_tp_last_error()
+
+
+def test_accurate_mode_is_zero():
+    """A caller that passes 0 (or zero-initialised options) gets the mode that
+    meets the parity bar on every tested workload."""
+    assert binding.ACCURATE == 0 and binding.FAST == binding.FAST_FC2_FORWARD | binding.FAST_FC1_BACKWARD_DATA
+    text = open(HEADER).read()
+    assert "MLP_TP_ACCURATE = 0" in text
 
 
 C_CLIENT = r"""

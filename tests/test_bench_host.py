@@ -78,3 +78,78 @@ def test_traffic_lookup(monkeypatch):
 def test_kernel_source_digest_covers_the_kernel_files():
     d = bench.kernel_source_digest()
     assert len(d) == 12 and int(d, 16) >= 0
+
+
+# ------------------------------------------------------------------ roofline arithmetic
+PEAKS = {"bf16_tflops": 1713.1, "bf16_tflops_sustained": 1430.5, "hbm_gbs": 6425.6}
+H4096 = dict(T=4096, h=4096, f=16384)
+
+
+def _stages(dom_ms, dom="fc1_backward_weight"):
+    ms = {s: 0.4 for s in bench.STAGES}
+    ms[dom] = dom_ms
+    return ms
+
+
+def test_roofline_counts_algorithmic_flops_of_one_gemm():
+    # the dA stage at 0.6944 ms, full clock: one GEMM of 2*T*h*f = 5.498e11 FLOPs
+    clocks = {"sm_mhz": 1957.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    r = bench.roofline_entry(_stages(0.6944), bench.MODES["fast"], clocks=clocks, peaks=PEAKS, peak_src="measured",
+                             **H4096)
+    assert r["stage"] == "fc1_backward_weight"
+    assert abs(r["algorithmic_flops_per_launch"] - 2 * 4096 * 4096 * 16384) < 1
+    assert abs(r["achieved"] - 791.7) < 1.0
+    # the power-cap bit alone does not switch the peak: the clock was at its maximum
+    assert r["peak"] == 1713.1 and abs(r["frac"] - 0.462) < 0.002
+    # both halves of the pair run: the executed tensor rate counts two products
+    assert r["executed_tensor_products"] == 2 and abs(r["executed_tflops"] - 2 * r["achieved"]) < 1e-6
+
+
+def test_roofline_takes_the_sustained_peak_only_when_the_clock_sagged():
+    low = {"sm_mhz": 1400.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    r = bench.roofline_entry(_stages(0.8), 0, clocks=low, peaks=PEAKS, peak_src="measured", **H4096)
+    assert r["peak"] == 1430.5
+    near = {"sm_mhz": 1920.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.roofline_entry(_stages(0.8), 0, clocks=near, peaks=PEAKS, peak_src="measured",
+                                **H4096)["peak"] == 1713.1
+    unsampled = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+    assert bench.roofline_entry(_stages(0.8), 0, clocks=unsampled, peaks=PEAKS, peak_src="measured",
+                                **H4096)["peak"] == 1713.1
+
+
+def test_roofline_fraction_stays_below_one_while_the_executed_rate_does():
+    """achieved counts one GEMM, the kernel runs one or two products: as long
+    as the executed tensor rate is within the peak, frac <= 1."""
+    for mode in (0, 3):
+        for clocks in ({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}, {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0}):
+            for dom_ms in (0.66, 0.7, 0.8, 1.2):
+                r = bench.roofline_entry(_stages(dom_ms), mode, clocks=clocks, peaks=PEAKS, peak_src="measured",
+                                         **H4096)
+                if r["executed_frac_of_peak"] <= 1.0:
+                    assert r["frac"] <= 1.0, r
+
+
+def test_stage_products_follow_the_mode():
+    acc, fast = bench.stage_products(bench.MODES["accurate"]), bench.stage_products(bench.MODES["fast"])
+    assert sum(acc.values()) == 10 and sum(fast.values()) == 8
+    assert acc["fc2_forward"] == acc["fc1_backward_data"] == 2 and fast["fc2_forward"] == fast["fc1_backward_data"] == 1
+
+
+def test_auto_mode_is_fast_only_where_its_parity_test_passes():
+    assert bench.pick_mode("auto", "h4096") == "fast"
+    assert bench.pick_mode("auto", "8.3b-class") == "accurate"
+    assert bench.pick_mode("accurate", "h4096") == "accurate"
+
+
+def test_clock_summary_keeps_only_samples_inside_the_window():
+    import datetime
+    txt = "\n".join([
+        "2026/12/03 05:28:00.100, 0, 1965, 1965, 300.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 05:28:00.200, 0, 1500, 1965, 900.5, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 05:28:00.300, 0, 1400, 1965, 950.5, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 05:28:00.400, 0, 1965, 1965, 200.5, 0x0, Not Active, Not Active, Not Active, Not Active"])
+    t0, t1 = datetime.datetime(2026, 12, 3, 5, 28, 0, 150000), datetime.datetime(2026, 12, 3, 5, 28, 0, 350000)
+    c = bench.summarize_clocks(txt, t0, t1)
+    assert c["samples"] == 2 and c["sm_mhz"] == 1450.0 and c["reasons"] == ["sw_power_cap"]
+    assert bench.summarize_clocks(txt)["samples"] == 4
+    assert bench.summarize_clocks("")["reasons"] == ["unsampled"]

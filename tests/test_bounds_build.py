@@ -30,11 +30,11 @@ binding.LIB_PATH = sys.argv[2]
 from oracle import mlp_oracle as oracle
 from tensor_transformer_mlp_bias_b200 import block, inputs
 from tests.parity_util import assert_close, to_gpu
-shapes = [(333, 320, 1280, 5, 0), (1024, 256, 1024, 2, 0), (2048, 128, 512, 4, 3), (1, 64, 128, 2, 0),
-          (257, 512, 768, 3, 3)]
-for T, h, f, t, split in shapes:
+shapes = [(333, 320, 1280, 5, 3), (1024, 256, 1024, 2, 3), (2048, 128, 512, 4, 0), (1, 64, 128, 2, 3),
+          (257, 512, 768, 3, 0)]
+for T, h, f, t, mode in shapes:
     inp = inputs.make_custom(T, h, f, seed=T + f)
-    out = block.forward_backward(to_gpu(inp), t, split=split)  # mlp_tp_check raises on MLP_ERR_BOUNDS
+    out = block.forward_backward(to_gpu(inp), t, mode=mode)  # mlp_tp_check raises on MLP_ERR_BOUNDS
     ref = oracle.full(inp)
     for k in ("Y", "dX", "dA", "da", "dB", "db"):
         assert_close(k, out[k], ref[k])
@@ -61,7 +61,7 @@ T, h = 4096, 1024
 dY = to_gpu(inputs.make_custom(T, h, 256, seed=3))["dY"]
 db = torch.empty(h, dtype=torch.bfloat16, device="cuda")  # h elements, as the call writes
 binding.mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db)
-torch.cuda.synchronize()
+binding.mlp_tp_check(None)  # the allocation-free path's own status word: raises on MLP_ERR_BOUNDS
 assert_close("db (allocation-free)", db, dY.double().sum(0).cpu().numpy())
 print("bounds-checked build: clean")
 """

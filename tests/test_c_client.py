@@ -86,8 +86,8 @@ int main(int argc, char** argv) {
   CK(cudaMemset(ws, 0, ws_bytes));
   cudaStream_t s;
   CK(cudaStreamCreate(&s));
-  MK(mlp_tp_forward(X, A, a, B, b, T, h, f, t, MLP_TP_SPLIT_NONE, Y, Z, H, H_lo, ws, ws_bytes, s));
-  MK(mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, MLP_TP_SPLIT_NONE, dX, dA, da, dB, db, ws, ws_bytes, s));
+  MK(mlp_tp_forward(X, A, a, B, b, T, h, f, t, MLP_TP_ACCURATE, Y, Z, H, H_lo, ws, ws_bytes, s));
+  MK(mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, MLP_TP_ACCURATE, dX, dA, da, dB, db, ws, ws_bytes, s));
   MK(mlp_tp_check(ws, s));
   char p[4096];
   const char* names[] = {"Y", "Z", "H", "dX", "dA", "da", "dB", "db"};

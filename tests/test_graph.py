@@ -15,10 +15,10 @@ from tests.parity_util import bits
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("shape,split", [((64, 256, 1024, 2), binding.SPLIT_NONE),
-                                         ((333, 320, 1280, 5), binding.SPLIT_ALL)],
-                         ids=["tiny", "ragged_split_all"])
-def test_graph_replay_matches_eager(shape, split):
+@pytest.mark.parametrize("shape,mode", [((64, 256, 1024, 2), binding.FAST),
+                                        ((333, 320, 1280, 5), binding.ACCURATE)],
+                         ids=["tiny_fast", "ragged_accurate"])
+def test_graph_replay_matches_eager(shape, mode):
     T, h, f, t = shape
     inp = {k: v.cuda() for k, v in inputs.make_custom(T, h, f, seed=51).items()}
     out = block.alloc_outputs(T, h, f)
@@ -27,15 +27,15 @@ def test_graph_replay_matches_eager(shape, split):
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):  # warm up (kernel attributes, occupancy) outside the capture
-        block.forward(inp, t, out, ws, split)
-        block.backward(inp, t, out, ws, split)
+        block.forward(inp, t, out, ws, mode)
+        block.backward(inp, t, out, ws, mode)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
 
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        block.forward(inp, t, out, ws, split)
-        block.backward(inp, t, out, ws, split)
+        block.forward(inp, t, out, ws, mode)
+        block.backward(inp, t, out, ws, mode)
 
     for seed in (52, 53):
         fresh = inputs.make_custom(T, h, f, seed=seed)
@@ -44,7 +44,7 @@ def test_graph_replay_matches_eager(shape, split):
         g.replay()
         torch.cuda.synchronize()
         binding.mlp_tp_check(ws)
-        eager = block.forward_backward({k: v.clone() for k, v in inp.items()}, t, split=split)
+        eager = block.forward_backward({k: v.clone() for k, v in inp.items()}, t, mode=mode)
         for k in ("Y", "Z", "H", "H_lo", "dX", "dA", "da", "dB", "db"):
             a, b = out[k], eager[k]
             same = torch.equal(a, b) if a.dtype == torch.float32 else torch.equal(bits(a), bits(b))

@@ -3,7 +3,12 @@
 Small shapes (several tiles, ragged tails) are compared element by element
 against the full oracle.  The five named workloads run at full size in the
 launch configuration the benchmark uses; the two smaller ones are compared in
-full, the three large ones at oracle-exact sampled rows and ffn indices.
+full, the three large ones at oracle-exact sampled rows and ffn indices that
+reach every output tile (parity_util.sample_indices).
+
+Every workload runs in the default precision mode (the low half of the
+activation pair in every product).  The fast mode (Y and dX from the high
+half only) runs on the workloads where the header says it meets the bar.
 
 Bar (elementwise, every output): max |gpu − oracle| ≤ 1e-2·(|oracle| + 1).
 """
@@ -15,15 +20,15 @@ import torch
 
 from oracle import mlp_oracle as oracle
 from tensor_transformer_mlp_bias_b200 import binding, block, inputs
-from tests.parity_util import assert_close, bits, to_gpu
+from tests.parity_util import FFN_GROUP, ROW_GROUP, assert_close, bits, sample_indices, to_gpu
 
 pytestmark = pytest.mark.gpu
 
-NONE, ALL = binding.SPLIT_NONE, binding.SPLIT_ALL
+ACCURATE, FAST = binding.ACCURATE, binding.FAST
 
 
-def run_all(inp_gpu, t, split=NONE):
-    out = block.forward_backward(inp_gpu, t, split=split)
+def run_all(inp_gpu, t, mode=None):
+    out = block.forward_backward(inp_gpu, t) if mode is None else block.forward_backward(inp_gpu, t, mode=mode)
     torch.cuda.synchronize()
     return out
 
@@ -49,13 +54,13 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("split", [NONE, ALL], ids=["split_none", "split_all"])
+@pytest.mark.parametrize("mode", [ACCURATE, FAST], ids=["accurate", "fast"])
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "T%d_h%d_f%d_t%d" % s)
-def test_small_shapes_full_oracle(shape, split):
+def test_small_shapes_full_oracle(shape, mode):
     T, h, f, t = shape
     inp = inputs.make_custom(T, h, f, seed=T + h + f + t)
     ref = oracle.full(inp)
-    check_full(run_all(to_gpu(inp), t, split), ref)
+    check_full(run_all(to_gpu(inp), t, mode), ref)
 
 
 def test_tiny_workload_every_divisor():
@@ -65,6 +70,7 @@ def test_tiny_workload_every_divisor():
     g = to_gpu(inp)
     for t in (1, 2, 4, 8, 16):
         check_full(run_all(g, t), ref)
+        check_full(run_all(g, t, FAST), ref)
 
 
 def test_empty_token_batch():
@@ -95,15 +101,27 @@ def test_gpt2_medium_full_oracle(t):
     check_full(run_all(to_gpu(inp), t), ref)
 
 
-def _sampled(name, t, split, n_rows, n_cols):
+def test_gpt2_medium_fast_mode():
+    inp, ref = _gpt2_medium()
+    check_full(run_all(to_gpu(inp), 8, FAST), ref)
+
+
+@functools.lru_cache(maxsize=1)
+def _sampled_reference(name):
+    """Inputs, sampled indices and the oracle's exact values there; the ffn
+    indices include both edges of every shard for each shard count the
+    workload lists."""
     wl = inputs.WORKLOADS[name]
     inp = inputs.make_inputs(wl)
-    out = run_all(to_gpu(inp), t, split)
     rng = np.random.default_rng(1234)
-    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, n_rows, replace=False)]))
-    cols = np.unique(np.concatenate([[0, wl.f - 1], rng.choice(wl.f, n_cols, replace=False)]))
-    sr = oracle.sample_rows(inp, rows)
-    sc = oracle.sample_ffn(inp, cols)
+    rows = sample_indices(wl.T, ROW_GROUP, rng)
+    cols = np.unique(np.concatenate([sample_indices(wl.f, FFN_GROUP, rng, wl.f // t) for t in wl.shards]))
+    return inp, rows, cols, oracle.sample_rows(inp, rows), oracle.sample_ffn(inp, cols)
+
+
+def _sampled(name, t, mode=None):
+    inp, rows, cols, sr, sc = _sampled_reference(name)
+    out = run_all(to_gpu(inp), t, mode)
     r = torch.as_tensor(rows, device="cuda")
     c = torch.as_tensor(cols, device="cuda")
     assert_close("Y rows", out["Y"][r], sr["Y"])
@@ -119,16 +137,26 @@ def _sampled(name, t, split, n_rows, n_cols):
 
 @pytest.mark.parametrize("t", [1, 4, 8])
 def test_h4096_sampled(t):
-    _sampled("h4096", t, NONE, 96, 96)
+    _sampled("h4096", t)
+
+
+@pytest.mark.parametrize("t", [1, 4, 8])
+def test_h4096_fast_mode_sampled(t):
+    """The bench's headline configuration: Y and dX from the high half."""
+    _sampled("h4096", t, FAST)
 
 
 def test_8p3b_class_sampled():
-    # sqrt(f)·|B| is largest here: Y and dX need the (hi, lo) activation pair too
-    _sampled("8.3b-class", 8, ALL, 64, 64)
+    # sqrt(f)·|B| is largest here: Y and dX need the low half of the pair, which the default mode uses
+    _sampled("8.3b-class", 8)
 
 
 def test_175b_class_sampled():
-    _sampled("175b-class", 8, NONE, 32, 32)
+    _sampled("175b-class", 8)
+
+
+def test_175b_class_fast_mode_sampled():
+    _sampled("175b-class", 8, FAST)
 
 
 # ------------------------------------------------------------------ invariants with no oracle
@@ -153,21 +181,21 @@ def test_t_independence_and_determinism():
         assert torch.equal(a, b) if a.dtype == torch.float32 else torch.equal(bits(a), bits(b)), k
 
 
-@pytest.mark.parametrize("split", [NONE, ALL], ids=["split_none", "split_all"])
-def test_stage_entry_points_match_composite(split):
+@pytest.mark.parametrize("mode", [ACCURATE, FAST], ids=["accurate", "fast"])
+def test_stage_entry_points_match_composite(mode):
     T, h, f, t = 300, 256, 1024, 4
     inp = to_gpu(inputs.make_custom(T, h, f, seed=9))
-    comp = run_all(inp, t, split)
+    comp = run_all(inp, t, mode)
     ws = binding.make_workspace(T, h, f, t)
     e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
     Z = torch.empty(T, f, dtype=torch.float32, device="cuda")
     H, H_lo, Y, dH, dH_lo = e(T, f), e(T, f), e(T, h), e(T, f), e(T, f)
     dX, dA, dB, da, db = e(T, h), e(h, f), e(f, h), e(f), e(h)
     binding.mlp_tp_fc1_forward(inp["X"], inp["A"], inp["a"], T, h, f, t, Z, H, H_lo, ws)
-    binding.mlp_tp_fc2_forward(H, H_lo if split & 1 else None, inp["B"], inp["b"], T, h, f, t, Y, ws)
+    binding.mlp_tp_fc2_forward(H, None if mode & FAST else H_lo, inp["B"], inp["b"], T, h, f, t, Y, ws)
     binding.mlp_tp_fc2_backward_data(inp["dY"], inp["B"], Z, T, h, f, t, dH, dH_lo, da, ws)
     binding.mlp_tp_fc2_backward_weight(H, H_lo, inp["dY"], T, h, f, t, dB, db, ws)
-    binding.mlp_tp_fc1_backward_data(dH, dH_lo if split & 2 else None, inp["A"], T, h, f, t, dX, ws)
+    binding.mlp_tp_fc1_backward_data(dH, None if mode & FAST else dH_lo, inp["A"], T, h, f, t, dX, ws)
     binding.mlp_tp_fc1_backward_weight(inp["X"], dH, dH_lo, T, h, f, t, dA, ws)
     binding.mlp_tp_check(ws)
     for k, v in dict(H=H, H_lo=H_lo, Y=Y, dX=dX, dA=dA, dB=dB, da=da, db=db).items():
@@ -248,7 +276,7 @@ def test_large_preactivations_saturate_gelu():
     host["X"] = (host["X"].float() * 3.0).to(torch.bfloat16)
     ref = oracle.full(host)
     assert float(np.abs(ref["Z"]).max()) > 20.0
-    out = run_all(to_gpu(host), t, ALL)
+    out = run_all(to_gpu(host), t)
     for k in out:
         assert bool(torch.isfinite(out[k].float()).all()), k
     check_full(out, ref)

@@ -31,7 +31,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, shape, sp, split, results):
+def _worker(rank, world, port, shape, sp, mode, results):
     import torch.distributed as dist
     from oracle import mlp_oracle as oracle
     from tensor_transformer_mlp_bias_b200 import inputs
@@ -49,8 +49,8 @@ def _worker(rank, world, port, shape, sp, split, results):
         rows = tp.token_rows(T, rank, world) if sp else slice(0, T)
         X = d["X"][rows] if sp else d["X"]
         dY = d["dY"][rows] if sp else d["dY"]
-        Y, saved = tp.forward(X, A_i, a_i, B_i, d["b"], sequence_parallel=sp, split=split, ops=tp_cpu_ops)
-        g = tp.backward(dY, saved, A_i, B_i, sequence_parallel=sp, split=split, ops=tp_cpu_ops)
+        Y, saved = tp.forward(X, A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode, ops=tp_cpu_ops)
+        g = tp.backward(dY, saved, A_i, B_i, sequence_parallel=sp, mode=mode, ops=tp_cpu_ops)
         err = {
             "Y": np.abs(Y.numpy() - ref["Y"][rows]).max(),
             "dX": np.abs(g["dX"].numpy() - ref["dX"][rows]).max(),
@@ -65,12 +65,12 @@ def _worker(rank, world, port, shape, sp, split, results):
         dist.destroy_process_group()
 
 
-def _run(world, shape, sp, split):
+def _run(world, shape, sp, mode):
     ctx = mp.get_context("spawn")
     manager = ctx.Manager()
     results = manager.dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, shape, sp, split, results)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, shape, sp, mode, results)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -80,9 +80,9 @@ def _run(world, shape, sp, split):
 
 
 @pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
-@pytest.mark.parametrize("split", [0, 3], ids=["split_none", "split_all"])
-def test_two_ranks_match_the_unsharded_block(sp, split):
-    res = _run(2, (64, 128, 256), sp, split)
+@pytest.mark.parametrize("mode", [0, 3], ids=["accurate", "fast"])
+def test_two_ranks_match_the_unsharded_block(sp, mode):
+    res = _run(2, (64, 128, 256), sp, mode)
     assert set(res) == {0, 1}
     for rank, errs in res.items():
         for k, e in errs.items():

@@ -24,7 +24,7 @@ def _free_port():
     return port
 
 
-def _worker(port, sp, split, results):
+def _worker(port, sp, mode, results):
     import torch
     import torch.distributed as dist
     from oracle import mlp_oracle as oracle
@@ -41,8 +41,8 @@ def _worker(port, sp, split, results):
         ref = oracle.full(inp)
         d = {k: v.cuda() for k, v in inp.items()}
         A_i, a_i, B_i = tp.shard_parameters(d["A"], d["a"], d["B"], 0, 1)
-        Y, saved = tp.forward(d["X"], A_i, a_i, B_i, d["b"], sequence_parallel=sp, split=split)
-        g = tp.backward(d["dY"], saved, A_i, B_i, sequence_parallel=sp, split=split)
+        Y, saved = tp.forward(d["X"], A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode)
+        g = tp.backward(d["dY"], saved, A_i, B_i, sequence_parallel=sp, mode=mode)
         torch.cuda.synchronize()
         out = dict(g, Y=Y)
         results["ratios"] = {k: worst_ratio(out[k], ref[k]) for k in ("Y", "dX", "dA", "da", "dB", "db")}
@@ -51,12 +51,12 @@ def _worker(port, sp, split, results):
 
 
 @pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
-@pytest.mark.parametrize("split", [0, 3], ids=["split_none", "split_all"])
-def test_one_rank_through_the_library_meets_the_bar(sp, split):
+@pytest.mark.parametrize("mode", [0, 3], ids=["accurate", "fast"])
+def test_one_rank_through_the_library_meets_the_bar(sp, mode):
     ctx = mp.get_context("spawn")
     manager = ctx.Manager()
     results = manager.dict()
-    p = ctx.Process(target=_worker, args=(_free_port(), sp, split, results))
+    p = ctx.Process(target=_worker, args=(_free_port(), sp, mode, results))
     p.start()
     p.join(300)
     assert p.exitcode == 0
