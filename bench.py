@@ -330,6 +330,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="h4096")
     ap.add_argument("--t", type=int, default=None)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (small profiling captures of the large workloads; "
+                         "the headline uses the workload's own T)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--mode", default="auto", choices=["auto", "fast", "accurate"],
                     help="precision mode: accurate (library default: Y and dX over the bf16 pair), fast (Y and dX "
@@ -349,6 +352,9 @@ def main():
 
     from tensor_transformer_mlp_bias_b200 import inputs
     wl = inputs.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, T=args.tokens)
     if args.t is None:
         args.t = max(wl.shards)
     world, rank, local = dist_env()
@@ -680,7 +686,7 @@ def main():
     # ------------------------------------------------ roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     roofline = roofline_entry(stage_ms, mode, T, h, f, clk_stages.summary(), peaks, peak_src)
-    roofline["traffic"] = traffic_for(roofline["stage"], wl, t)
+    roofline["traffic"] = traffic_for(roofline["stage"], wl, t) if args.tokens is None else None
     products = stage_products(mode)
     clocks = clk.summary()
     peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -761,7 +767,7 @@ def traffic_for(stage, wl, t):
 def kernel_source_digest():
     import hashlib
     hsh = hashlib.sha256()
-    for n in ("gemm.cuh", "ptx.cuh", "colsum.cuh", "mlp_tp.cu"):
+    for n in ("gemm.cuh", "ptx.cuh", "colsum.cuh", "peer.cuh", "peer_reduce.cuh", "mlp_tp.cu"):
         with open(os.path.join(ROOT, "tensor_transformer_mlp_bias_b200", "csrc", n), "rb") as fh:
             hsh.update(fh.read())
     return hsh.hexdigest()[:12]

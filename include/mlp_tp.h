@@ -221,6 +221,95 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
                                        void* dX, void* dA, void* da, void* dB, void* db,
                                        void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------- across GPUs */
+
+/* The block sharded over `world` GPUs, one shard per GPU (rank r holds
+ * columns [r·f/world, (r+1)·f/world) of A and a and those rows of B; each
+ * rank calls the stage entry points above with t = 1 on its shard, fs =
+ * f/world).  The two sums of the tensor-parallel pair ("Megatron-LM — 架构与
+ * 原理", §4 巧妙之处: Y = Σ_r P_r + b after the row-parallel layer, the
+ * reduce operator's forward all-reduce, and dX = Σ_r Q_r, the copy
+ * operator's backward all-reduce) are fused into the row-parallel GEMMs:
+ *
+ *  - mlp_tp_fc2_forward_peer / mlp_tp_fc1_backward_data_peer compute this
+ *    rank's partial P_r = (H_r + H_lo_r)·B_r (or Q_r = (dH_r + dH_lo_r)·A_rᵀ)
+ *    in fp32 and, from the GEMM epilogue, store each 128-row block of it into
+ *    the receive buffer of the rank that owns those tokens (rank o owns rows
+ *    [o·T/world, (o+1)·T/world)), slot r, with plain stores through the peer
+ *    mapping (NVLink), then raise that block's arrival count on the owner;
+ *  - mlp_tp_peer_reduce, on the owner, waits for the `world` partials of each
+ *    block, sums them in fp32 in rank order, adds `bias` once (NULL: none),
+ *    rounds once to bf16 into out[T/world, h] (this rank's token rows) and
+ *    marks the block consumed, so the next exchange may overwrite it.
+ *
+ * That is the reduce-scatter of the sequence-parallel form; the plain
+ * tensor-parallel form follows it with an all-gather of the bf16 rows.  The
+ * partials stay fp32 and are rounded once: summing per-rank bf16 outputs,
+ * as a 16-bit all-reduce does, exceeds 1e-2·(|exact| + 1) on the 8.3B-class
+ * workload at 2, 4 and 8 ranks.
+ *
+ * Buffers.  Each rank allocates (device memory, zero-filled once) a receive
+ * buffer of mlp_tp_peer_recv_bytes(T, h, world) bytes ([world][T/world][h]
+ * fp32) and a flag block of mlp_tp_peer_flag_bytes(T, h, world) bytes, and
+ * every rank's descriptor lists all ranks' buffers as addressed from its own
+ * GPU (its own pointers for itself; mappings of the others', for example
+ * from mlp_tp_ipc_import).  Shapes: T % world == 0, and with world > 1 the
+ * T/world rows of a rank a multiple of 128; h as elsewhere.
+ *
+ * Ordering.  `epoch` numbers the exchanges on these buffers: 1 for the first,
+ * then +1 per exchange, the same on every rank.  Each wait is bounded by the
+ * wait budget (mlp_tp_set_wait_budget_ns); one that runs out records
+ * MLP_ERR_TIMEOUT in the caller's workspace (mlp_tp_check), and the flag
+ * blocks must then be zero-filled again and `epoch` restarted at 1.  With
+ * epoch == 0 no flag is read or written (flags may be NULL): the caller
+ * orders the GEMM and the reduce itself, e.g. on one stream with a
+ * collective on the fp32 buffer in between (world = 1 then describes this
+ * rank's own buffer: the GEMM writes its whole [T, h] partial to slot 0). */
+#define MLP_TP_MAX_WORLD 8
+#define MLP_TP_IPC_HANDLE_BYTES 64
+
+typedef struct {
+  int32_t rank;                   /* this GPU's rank, 0 <= rank < world */
+  int32_t world;                  /* GPUs in the group, 1..MLP_TP_MAX_WORLD */
+  uint32_t epoch;                 /* exchange number (1, 2, ...), or 0: no flags */
+  uint32_t reserved;              /* 0 */
+  void* recv[MLP_TP_MAX_WORLD];   /* rank o's receive buffer as addressed from this GPU */
+  void* flags[MLP_TP_MAX_WORLD];  /* rank o's flag block as addressed from this GPU */
+} mlp_tp_peer_t;
+
+/* Bytes of one rank's receive buffer and flag block (multiples of 256);
+ * 0 for an invalid shape. */
+size_t mlp_tp_peer_recv_bytes(int64_t T, int64_t h, int32_t world);
+size_t mlp_tp_peer_flag_bytes(int64_t T, int64_t h, int32_t world);
+
+/* This rank's row-parallel partial P_r = (H + H_lo)·B (H_lo NULL: H only),
+ * H[T, fs], B[fs, h], sent to the owners as described above.  `ws` as for
+ * mlp_tp_fc2_forward with f = fs, t = 1. */
+mlp_status_t mlp_tp_fc2_forward_peer(const void* H, const void* H_lo, const void* B,
+                                     int64_t T, int64_t h, int64_t fs, const mlp_tp_peer_t* peer,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* This rank's partial input gradient Q_r = (dH + dH_lo)·Aᵀ (dH_lo NULL: dH
+ * only), dH[T, fs], A[h, fs], sent to the owners likewise. */
+mlp_status_t mlp_tp_fc1_backward_data_peer(const void* dH, const void* dH_lo, const void* A,
+                                           int64_t T, int64_t h, int64_t fs, const mlp_tp_peer_t* peer,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+/* The owner's sum: out[T/world, h] = bf16(Σ_r slot r + bias), rank order.
+ * `ws` needs only its 256-byte status header here. */
+mlp_status_t mlp_tp_peer_reduce(const mlp_tp_peer_t* peer, const void* bias, int64_t T, int64_t h,
+                                void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Mapping a buffer of another process on another GPU (CUDA IPC).
+ * mlp_tp_ipc_export writes the MLP_TP_IPC_HANDLE_BYTES-byte handle of the
+ * allocation that holds `ptr` and ptr's offset in it; mlp_tp_ipc_import, in
+ * another process, maps that allocation (peer access enabled) and returns
+ * the address of the same byte; mlp_tp_ipc_close unmaps it.  A process does
+ * not import its own handles. */
+mlp_status_t mlp_tp_ipc_export(const void* ptr, void* handle, uint64_t* offset);
+mlp_status_t mlp_tp_ipc_import(const void* handle, uint64_t offset, void** ptr);
+mlp_status_t mlp_tp_ipc_close(void* ptr, uint64_t offset);
+
 /* ----------------------------------------------------- allocation-free */
 
 /* db = sum over rows of dY (the row-parallel layer's bias gradient, as

@@ -33,6 +33,19 @@ _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I32 = ctypes.c_int32
 _SZ = ctypes.c_size_t
+
+MAX_WORLD = 8
+IPC_HANDLE_BYTES = 64
+
+
+class Peer(ctypes.Structure):
+    """mlp_tp_peer_t: one rank's view of the cross-GPU reduction buffers."""
+    _fields_ = [("rank", ctypes.c_int32), ("world", ctypes.c_int32), ("epoch", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32), ("recv", ctypes.c_void_p * MAX_WORLD),
+                ("flags", ctypes.c_void_p * MAX_WORLD)]
+
+
+_PP = ctypes.POINTER(Peer)
 _SIGS = {
     "mlp_tp_workspace_bytes": ([_I64, _I64, _I64, _I32], _SZ),
     "mlp_tp_forward": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 4 + [_P, _SZ, _P], ctypes.c_int),
@@ -47,6 +60,14 @@ _SIGS = {
     "mlp_tp_forward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_backward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 5 + [_P, _SZ, _P],
                                   ctypes.c_int),
+    "mlp_tp_peer_recv_bytes": ([_I64, _I64, _I32], _SZ),
+    "mlp_tp_peer_flag_bytes": ([_I64, _I64, _I32], _SZ),
+    "mlp_tp_fc2_forward_peer": ([_P] * 3 + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_data_peer": ([_P] * 3 + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_peer_reduce": ([_PP, _P, _I64, _I64, _P, _P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_ipc_export": ([_P, _P, ctypes.POINTER(ctypes.c_uint64)], ctypes.c_int),
+    "mlp_tp_ipc_import": ([_P, ctypes.c_uint64, ctypes.POINTER(_P)], ctypes.c_int),
+    "mlp_tp_ipc_close": ([_P, ctypes.c_uint64], ctypes.c_int),
     "mlp_tp_fc2_bias_grad_noalloc": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "mlp_tp_check": ([_P, _P], ctypes.c_int),
     "mlp_tp_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -226,6 +247,73 @@ def mlp_tp_backward_recompute(dY, X, A, a, B, T, h, f, t, mode, dX, dA, da, dB, 
                                            _addr(a, "a"), _addr(B, "B"), T, h, f, t, mode,
                                            _addr(dX, "dX", T == 0), _addr(dA, "dA"), _addr(da, "da", True),
                                            _addr(dB, "dB"), _addr(db, "db", True), w, wn, _stream(stream)))
+
+
+# ------------------------------------------------------------------ across GPUs
+def _ptr(x):
+    if x is None:
+        return None
+    return x if isinstance(x, int) else x.data_ptr()
+
+
+def make_peer(rank: int, world: int, recv, flags=None, epoch: int = 0) -> Peer:
+    """mlp_tp_peer_t for rank `rank` of `world`: recv[o] and flags[o] are rank
+    o's receive buffer and flag block as addressed from this GPU (ints or
+    tensors; flags may be None when epoch == 0)."""
+    if not 1 <= world <= MAX_WORLD or not 0 <= rank < world or len(recv) != world:
+        raise ValueError(f"peer table: rank {rank} of {world} with {len(recv)} buffers")
+    p = Peer()
+    p.rank, p.world, p.epoch, p.reserved = rank, world, epoch, 0
+    for o in range(world):
+        p.recv[o] = _ptr(recv[o])
+        p.flags[o] = _ptr(flags[o]) if flags is not None else None
+    return p
+
+
+def peer_recv_bytes(T: int, h: int, world: int) -> int:
+    return int(lib().mlp_tp_peer_recv_bytes(T, h, world))
+
+
+def peer_flag_bytes(T: int, h: int, world: int) -> int:
+    return int(lib().mlp_tp_peer_flag_bytes(T, h, world))
+
+
+def mlp_tp_fc2_forward_peer(H, H_lo, B, T, h, fs, peer: Peer, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_forward_peer(_addr(H, "H", T == 0), _addr(H_lo, "H_lo", True), _addr(B, "B"), T, h, fs,
+                                         ctypes.byref(peer), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_data_peer(dH, dH_lo, A, T, h, fs, peer: Peer, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_data_peer(_addr(dH, "dH", T == 0), _addr(dH_lo, "dH_lo", True), _addr(A, "A"),
+                                               T, h, fs, ctypes.byref(peer), w, wn, _stream(stream)))
+
+
+def mlp_tp_peer_reduce(peer: Peer, bias, T, h, out, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_peer_reduce(ctypes.byref(peer), _addr(bias, "bias", True), T, h,
+                                    _addr(out, "out", T == 0), w, wn, _stream(stream)))
+
+
+def mlp_tp_ipc_export(ptr) -> tuple:
+    """(handle bytes, offset) of the device allocation holding `ptr`."""
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    _check(lib().mlp_tp_ipc_export(_ptr(ptr), handle, ctypes.byref(off)))
+    return handle.raw, int(off.value)
+
+
+def mlp_tp_ipc_import(handle: bytes, offset: int) -> int:
+    """Address, in this process, of the byte another process exported."""
+    out = ctypes.c_void_p(0)
+    buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    _check(lib().mlp_tp_ipc_import(buf, offset, ctypes.byref(out)))
+    return int(out.value)
+
+
+def mlp_tp_ipc_close(ptr: int, offset: int):
+    _check(lib().mlp_tp_ipc_close(ptr, offset))
 
 
 def mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db, stream=None):

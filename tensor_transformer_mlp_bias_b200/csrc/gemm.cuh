@@ -50,6 +50,12 @@
 // 64 (rows) x 64 (K); the MMA reads it through an MN-major descriptor, so no
 // transpose is ever materialised.
 //
+// Cross-GPU shard reduction (EPI_PEER).  With the block sharded over several
+// GPUs, a rank's row-parallel GEMM sends each 128-row block of its fp32
+// partial straight to the GPU that owns those token rows (peer.cuh): plain
+// coalesced stores over NVLink from the epilogue, then a per-tile arrival
+// count raised at system scope; the owner's reduce kernel sums the partials.
+//
 // Every wait is bounded (see mbar_wait).  A wait that runs out records
 // status 7 (timeout) in the device status word, raises a CTA-wide abort
 // flag so the other roles leave their loops, and the CTA still drains its
@@ -60,6 +66,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "peer.cuh"
 #include "ptx.cuh"
 
 namespace mlptp {
@@ -72,7 +79,7 @@ constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int CTL_BYTES = 1024;
 
-enum Epi : int { EPI_BIAS_GELU = 0, EPI_SHARD_SUM = 1, EPI_GELU_GRAD = 2, EPI_STORE = 3 };
+enum Epi : int { EPI_BIAS_GELU = 0, EPI_SHARD_SUM = 1, EPI_GELU_GRAD = 2, EPI_STORE = 3, EPI_PEER = 4 };
 
 // Epilogue staging per epilogue warp: one 32x32 tile per output, laid out
 // for the TMA store (bf16: 64-byte rows, 64-byte swizzle; fp32: 128-byte
@@ -81,7 +88,8 @@ constexpr int EPI_BF16_TILE = 32 * 32 * 2;
 constexpr int EPI_F32_TILE = 32 * 32 * 4;
 __host__ __device__ constexpr int epi_warp_bytes(int epi) {
   return epi == EPI_BIAS_GELU ? EPI_F32_TILE + 2 * EPI_BF16_TILE
-                              : (epi == EPI_GELU_GRAD ? 2 * EPI_BF16_TILE : EPI_BF16_TILE);
+                              : (epi == EPI_GELU_GRAD ? 2 * EPI_BF16_TILE
+                                                      : (epi == EPI_PEER ? EPI_F32_TILE : EPI_BF16_TILE));
 }
 
 // Tile shape.  TN is the number of output columns per tile: 256 (one MMA
@@ -172,6 +180,8 @@ struct GemmParams {
   unsigned int* status;       // device status word pair in the workspace
   unsigned long long budget_ns;
   unsigned int debug_flags;
+  PeerParams peer;            // EPI_PEER: where each row block's partial goes
+  long long peer_recv_elems;  // floats in each receive buffer (bounds-checking build)
 };
 
 // Tensor maps of the operands, one per K part (part 1 repeats part 0 for an
@@ -394,6 +404,8 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
   using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   static_assert(!DUAL || PAIR, "both halves of A in one stage: pair mode");
   static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
+  static_assert(EPI != EPI_PEER || (TN == 256 && EW == PEER_ARRIVALS),
+                "a peer tile block is one MMA width and its arrival count is one per epilogue warp");
   constexpr int ACCS = Cfg::ACCS;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -669,6 +681,28 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
       float sum[EPI == EPI_SHARD_SUM ? SLICE_COLS : 1];
+      // EPI_PEER: the rank that owns this CTA's 128 token rows, the block's
+      // index in that rank's buffers, and (with flags) the wait for the
+      // owner to have consumed the previous exchange's values in this slot
+      int peer_owner = 0, peer_lb = 0;
+      bool peer_blk = false;
+      if constexpr (EPI == EPI_PEER) {
+        peer_blk = row_block * BM < p.M;
+        if (peer_blk) {
+          peer_owner = p.peer.world == 1 ? 0 : (row_block * BM) / p.peer.rows;
+          peer_lb = row_block - peer_owner * (p.peer.rows / BM);
+          if (p.peer.epoch != 0u) {
+            if (lane == 0 &&
+                !peer_wait_at_least(peer_consumed(p.peer, peer_owner, peer_lb, nb), p.peer.epoch - 1u, budget))
+              record_timeout(p, abort_flag, 0x800u);
+            __syncwarp();
+            if (*abort_flag) {
+              ok = false;
+              break;
+            }
+          }
+        }
+      }
       for (int s = it.s_begin; s < it.s_end; ++s, ++unit) {
         const uint32_t acc = unit % ACCS, acc_phase = (unit / ACCS) & 1u;
         // bias+GeLU on wide tiles (single accumulator, epilogue not hidden):
@@ -748,6 +782,29 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
               const long long ci = static_cast<long long>(row_block * 4 + q) * p.N + col + lane;
               if (index_ok(ci, p.colsum_elems, p.status, 0x501u)) p.colsum[ci] = cs;
             }
+          } else if constexpr (EPI == EPI_PEER) {
+            // this warp's 32 rows x 32 columns of the fp32 partial, into
+            // slot `rank` of the owner's receive buffer: transposed through
+            // the staging tile so 8 lanes write each 128-byte row segment
+            if (peer_blk) {
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+              stage_f32x32(st_f32, lane, v);
+              __syncwarp();
+              const long long base =
+                  (static_cast<long long>(p.peer.rank) * p.peer.rows + (row0 - peer_owner * p.peer.rows)) * p.N + col;
+              float* dst = p.peer.recv[peer_owner];
+              const int rr = lane >> 3, cc = lane & 7;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int rw = i * 4 + rr;
+                const long long di = base + static_cast<long long>(rw) * p.N + cc * 4;
+                if (row0 + rw < p.M && index_ok(di + 3, p.peer_recv_elems, p.status, 0x509u))
+                  st_global_v4f(dst + di, ld_shared_v4f(st_f32 + rw * 128 + ((cc ^ (rw & 7)) << 4)));
+              }
+              __syncwarp();
+            }
           } else if constexpr (EPI == EPI_STORE) {
             if (it.piece >= 0) {
               // one K piece of a split tile: its fp32 sum goes to the scratch
@@ -822,6 +879,14 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
           } else {
             mbar_arrive(&ctl->tempty[acc]);
           }
+        }
+      }
+      if constexpr (EPI == EPI_PEER) {
+        // every lane's stores reach the owner before this warp's arrival does
+        if (ok && peer_blk && p.peer.epoch != 0u) {
+          __threadfence_system();
+          __syncwarp();
+          if (lane == 0) red_add_release_sys(peer_counter(p.peer, peer_owner, peer_lb, nb), 1u);
         }
       }
     }

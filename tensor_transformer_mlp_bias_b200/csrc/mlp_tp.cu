@@ -14,6 +14,7 @@
 #include "../../include/mlp_tp.h"
 #include "colsum.cuh"
 #include "gemm.cuh"
+#include "peer_reduce.cuh"
 
 using namespace mlptp;
 
@@ -377,7 +378,8 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   {
-    mlp_status_t st = make_out_map(&maps.out[0], p.out0, g.M, g.N, false, name);
+    // EPI_PEER stores with plain instructions and has no output tensor map
+    mlp_status_t st = p.out0 != nullptr ? make_out_map(&maps.out[0], p.out0, g.M, g.N, false, name) : MLP_OK;
     if (st == MLP_OK && p.out1 != nullptr) st = make_out_map(&maps.out[1], p.out1, g.M, g.N, false, name);
     if (st == MLP_OK && p.out_f32 != nullptr) st = make_out_map(&maps.out[2], p.out_f32, g.M, g.N, true, name);
     if (st != MLP_OK) return st;
@@ -671,6 +673,79 @@ mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, 
   return launch_gemm<true, true, EPI_STORE, kWideTN>(g, p, L, "column-parallel weight gradient (dA)");
 }
 
+// ---------------------------------------------------------------- across GPUs
+// Buffers and tile blocks of the cross-GPU shard reduction (peer.cuh).
+struct PeerShape {
+  int64_t rows, nbl, ncb;
+};
+
+PeerShape peer_shape(int64_t T, int64_t h, int32_t world) {
+  const int64_t rows = T / world;
+  return PeerShape{rows, (rows + PEER_BLOCK_ROWS - 1) / PEER_BLOCK_ROWS, (h + PEER_BLOCK_COLS - 1) / PEER_BLOCK_COLS};
+}
+size_t peer_recv_bytes(int64_t T, int64_t h) { return align_up(static_cast<size_t>(T * h) * sizeof(float), 256); }
+size_t peer_flag_bytes(const PeerShape& ps) {
+  return align_up(static_cast<size_t>(2 * ps.nbl * ps.ncb) * sizeof(unsigned int), 256);
+}
+
+mlp_status_t check_peer(const mlp_tp_peer_t* peer, int64_t T, int64_t h, PeerParams& q, long long& recv_elems) {
+  if (peer == nullptr) return fail(MLP_ERR_INVALID_ARG, "peer descriptor is NULL");
+  const int32_t world = peer->world, rank = peer->rank;
+  if (world < 1 || world > MLP_TP_MAX_WORLD)
+    return fail(MLP_ERR_INVALID_ARG, "peer world %d outside 1..%d", world, MLP_TP_MAX_WORLD);
+  if (rank < 0 || rank >= world) return fail(MLP_ERR_INVALID_ARG, "peer rank %d outside 0..%d", rank, world - 1);
+  if (T % world != 0)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "T=%lld tokens do not split over %d ranks", (long long)T, world);
+  const PeerShape ps = peer_shape(T, h, world);
+  if (world > 1 && ps.rows % PEER_BLOCK_ROWS != 0)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "T/world=%lld token rows per rank must be a multiple of %d",
+                (long long)ps.rows, PEER_BLOCK_ROWS);
+  memset(&q, 0, sizeof(q));
+  for (int r = 0; r < world; ++r) {
+    if (peer->recv[r] == nullptr && T > 0) return fail(MLP_ERR_INVALID_ARG, "peer receive buffer %d is NULL", r);
+    if (reinterpret_cast<uintptr_t>(peer->recv[r]) % 16 != 0)
+      return fail(MLP_ERR_MISALIGNED, "peer receive buffer %d is not 16-byte aligned", r);
+    if (peer->epoch != 0u) {
+      if (peer->flags[r] == nullptr) return fail(MLP_ERR_INVALID_ARG, "peer flag block %d is NULL", r);
+      if (reinterpret_cast<uintptr_t>(peer->flags[r]) % 16 != 0)
+        return fail(MLP_ERR_MISALIGNED, "peer flag block %d is not 16-byte aligned", r);
+    }
+    q.recv[r] = static_cast<float*>(peer->recv[r]);
+    q.flags[r] = static_cast<unsigned int*>(peer->flags[r]);
+  }
+  q.rank = rank;
+  q.world = world;
+  q.rows = static_cast<int>(ps.rows);
+  q.nbl = static_cast<int>(ps.nbl);
+  q.ncb = static_cast<int>(ps.ncb);
+  q.epoch = peer->epoch;
+  recv_elems = static_cast<long long>(T) * h;
+  return MLP_OK;
+}
+
+mlp_status_t fc2_forward_peer(const Shape& s, const void* H, const void* H_lo, const void* B, const PeerParams& q,
+                              long long recv_elems, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.peer = q;
+  p.peer_recv_elems = recv_elems;
+  GemmDesc g{pair(H, H_lo, false), one(B, true), s.T, s.h, s.f, 1, H_lo != nullptr ? 2 : 1};
+  if (H_lo != nullptr)
+    return launch_gemm<false, true, EPI_PEER, 256, kPair, 8, kDualA>(g, p, L, "row-parallel forward to the owners (P)");
+  return launch_gemm<false, true, EPI_PEER>(g, p, L, "row-parallel forward to the owners (P)");
+}
+
+mlp_status_t fc1_backward_data_peer(const Shape& s, const void* dH, const void* dH_lo, const void* A,
+                                    const PeerParams& q, long long recv_elems, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.peer = q;
+  p.peer_recv_elems = recv_elems;
+  GemmDesc g{pair(dH, dH_lo, false), one(A, false), s.T, s.h, s.f, 1, dH_lo != nullptr ? 2 : 1};
+  if (dH_lo != nullptr)
+    return launch_gemm<false, false, EPI_PEER, 256, kPair, 8, kDualA>(g, p, L,
+                                                                     "column-parallel backward data to the owners (Q)");
+  return launch_gemm<false, false, EPI_PEER>(g, p, L, "column-parallel backward data to the owners (Q)");
+}
+
 // Common preamble: shape, pointers, workspace, device.
 mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, void* stream,
                       Launch& L, bool recompute = false) {
@@ -894,6 +969,117 @@ uint64_t mlp_tp_launch_count(void) { return g_launches.load(); }
 void mlp_tp_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
 void mlp_tp_set_debug_flags(uint32_t flags) { g_debug_flags.store(flags); }
+
+size_t mlp_tp_peer_recv_bytes(int64_t T, int64_t h, int32_t world) {
+  if (T < 0 || h < 64 || h % 64 != 0 || world < 1 || world > MLP_TP_MAX_WORLD || T % world != 0) return 0;
+  return peer_recv_bytes(T, h);
+}
+
+size_t mlp_tp_peer_flag_bytes(int64_t T, int64_t h, int32_t world) {
+  if (T < 0 || h < 64 || h % 64 != 0 || world < 1 || world > MLP_TP_MAX_WORLD || T % world != 0) return 0;
+  return peer_flag_bytes(peer_shape(T, h, world));
+}
+
+mlp_status_t mlp_tp_fc2_forward_peer(const void* H, const void* H_lo, const void* B, int64_t T, int64_t h, int64_t fs,
+                                     const mlp_tp_peer_t* peer, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, fs, 1};
+  Launch L;
+  PeerParams q;
+  long long recv_elems = 0;
+  mlp_status_t st = check_shape(s);
+  if (st != MLP_OK || (st = check_peer(peer, T, h, q, recv_elems)) != MLP_OK) return st;
+  st = prologue(s, {{H, "H", false, s.T == 0}, {H_lo, "H_lo", true, s.T == 0}, {B, "B", false}}, ws, ws_bytes, stream, L);
+  if (st != MLP_OK) return st;
+  return fc2_forward_peer(s, H, H_lo, B, q, recv_elems, ws, L);
+}
+
+mlp_status_t mlp_tp_fc1_backward_data_peer(const void* dH, const void* dH_lo, const void* A, int64_t T, int64_t h,
+                                           int64_t fs, const mlp_tp_peer_t* peer, void* ws, size_t ws_bytes,
+                                           void* stream) {
+  Shape s{T, h, fs, 1};
+  Launch L;
+  PeerParams q;
+  long long recv_elems = 0;
+  mlp_status_t st = check_shape(s);
+  if (st != MLP_OK || (st = check_peer(peer, T, h, q, recv_elems)) != MLP_OK) return st;
+  st = prologue(s, {{dH, "dH", false, s.T == 0}, {dH_lo, "dH_lo", true, s.T == 0}, {A, "A", false}}, ws, ws_bytes,
+                stream, L);
+  if (st != MLP_OK) return st;
+  return fc1_backward_data_peer(s, dH, dH_lo, A, q, recv_elems, ws, L);
+}
+
+mlp_status_t mlp_tp_peer_reduce(const mlp_tp_peer_t* peer, const void* bias, int64_t T, int64_t h, void* out,
+                                void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || h < 0) return fail(MLP_ERR_INVALID_ARG, "negative size T=%lld h=%lld", (long long)T, (long long)h);
+  if (h < 64 || h % 64 != 0 || T > (int64_t(1) << 31) - 1 || h > (int64_t(1) << 31) - 1)
+    return fail(MLP_ERR_UNSUPPORTED_SHAPE, "h=%lld must be a positive multiple of 64 and T, h < 2^31", (long long)h);
+  PeerParams q;
+  long long recv_elems = 0;
+  mlp_status_t st = check_peer(peer, T, h, q, recv_elems);
+  if (st != MLP_OK) return st;
+  if ((st = check_ptrs({{out, "out", false, q.rows == 0}, {bias, "bias", true}})) != MLP_OK) return st;
+  if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MLP_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+  if (ws_bytes < WS_HEADER_BYTES)
+    return fail(MLP_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, WS_HEADER_BYTES);
+  int dev = 0, sms = 0;
+  if ((st = current_device(dev, sms)) != MLP_OK) return st;
+  const long long blocks = static_cast<long long>(q.nbl) * q.ncb;
+  if (blocks == 0) return MLP_OK;
+  peer_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      q, static_cast<const __nv_bfloat16*>(bias), static_cast<int>(h), static_cast<__nv_bfloat16*>(out),
+      static_cast<unsigned int*>(ws), g_budget_ns.load(), recv_elems);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "peer_reduce");
+  g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+// ---- mapping another process's buffers (CUDA IPC)
+typedef CUresult (*GetAddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+mlp_status_t mlp_tp_ipc_export(const void* ptr, void* handle, uint64_t* offset) {
+  if (ptr == nullptr || handle == nullptr || offset == nullptr)
+    return fail(MLP_ERR_INVALID_ARG, "ipc export: NULL argument");
+  static GetAddressRangeFn range_fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      range_fn = reinterpret_cast<GetAddressRangeFn>(f);
+  });
+  if (range_fn == nullptr) return fail(MLP_ERR_CUDA, "cuMemGetAddressRange is unavailable");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  CUresult r = range_fn(&base, &size, reinterpret_cast<CUdeviceptr>(ptr));
+  if (r != CUDA_SUCCESS) return fail(MLP_ERR_CUDA, "cuMemGetAddressRange failed (CUresult %d)", (int)r);
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+  static_assert(sizeof(h) == MLP_TP_IPC_HANDLE_BYTES, "IPC handle size");
+  memcpy(handle, &h, sizeof(h));
+  *offset = static_cast<uint64_t>(reinterpret_cast<CUdeviceptr>(ptr) - base);
+  return MLP_OK;
+}
+
+mlp_status_t mlp_tp_ipc_import(const void* handle, uint64_t offset, void** ptr) {
+  if (handle == nullptr || ptr == nullptr) return fail(MLP_ERR_INVALID_ARG, "ipc import: NULL argument");
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+  *ptr = static_cast<char*>(base) + offset;
+  return MLP_OK;
+}
+
+mlp_status_t mlp_tp_ipc_close(void* ptr, uint64_t offset) {
+  if (ptr == nullptr) return fail(MLP_ERR_INVALID_ARG, "ipc close: NULL pointer");
+  cudaError_t e = cudaIpcCloseMemHandle(static_cast<char*>(ptr) - offset);
+  return e == cudaSuccess ? MLP_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
+}
 
 }  // extern "C"
 

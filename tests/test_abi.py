@@ -169,3 +169,57 @@ def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, (run.returncode, run.stderr)
     assert int(run.stdout.strip()) == binding.workspace_bytes(64, 256, 1024, 2)
+
+
+# ------------------------------------------------------------------ cross-GPU entry points (host side)
+def test_peer_buffer_sizes(lib):
+    # [world][T/world][h] fp32 receive buffer; two uint32 per (128-row block, 256-column block) of a rank
+    assert binding.peer_recv_bytes(4096, 4096, 8) == 4096 * 4096 * 4
+    assert binding.peer_flag_bytes(4096, 4096, 8) == 2 * 4 * 16 * 4   # 512 rows per rank: 4 blocks x 16
+    assert binding.peer_flag_bytes(4096, 4096, 1) == 2 * 32 * 16 * 4
+    assert binding.peer_recv_bytes(333, 320, 1) == (333 * 320 * 4 + 255) // 256 * 256
+    assert binding.peer_recv_bytes(100, 256, 3) == 0              # T not divisible by the ranks
+    assert binding.peer_recv_bytes(64, 96, 1) == 0                # h not a multiple of 64
+    assert binding.peer_flag_bytes(64, 256, 9) == 0               # more ranks than one NVLink group holds
+
+
+def _fc2_peer(lib, peer, T=512, h=256, fs=128):
+    import ctypes
+    return lib.mlp_tp_fc2_forward_peer(FAKE, None, FAKE, T, h, fs, None if peer is None else ctypes.byref(peer),
+                                       FAKE * 2, 1 << 30, None)
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (None, 1, "peer descriptor is NULL"),
+    (dict(world=9), 1, "world 9"),
+    (dict(rank=2, world=2), 1, "rank 2"),
+    (dict(world=3), 2, "do not split"),
+    (dict(world=2, T=640), 2, "multiple of 128"),
+    (dict(world=2, recv=[FAKE, None]), 1, "receive buffer 1 is NULL"),
+    (dict(world=2, recv=[FAKE, FAKE + 4]), 3, "receive buffer 1 is not 16-byte aligned"),
+    (dict(world=2, epoch=1, flags=None), 1, "flag block 0 is NULL"),
+])
+def test_peer_descriptor_is_validated_on_the_host(lib, kw, status, needle):
+    if kw is None:
+        st = _fc2_peer(lib, None)
+    else:
+        world = kw.get("world", 1)
+        recv = kw.get("recv", [FAKE] * world)
+        flags = kw.get("flags", [FAKE] * world)
+        peer = binding.Peer()
+        peer.rank, peer.world, peer.epoch = kw.get("rank", 0), world, kw.get("epoch", 0)
+        for o in range(min(world, binding.MAX_WORLD)):
+            peer.recv[o] = recv[o]
+            peer.flags[o] = flags[o] if flags is not None else None
+        st = _fc2_peer(lib, peer, T=kw.get("T", 512))
+    assert st == status, binding.mlp_tp_last_error()
+    assert needle in binding.mlp_tp_last_error()
+
+
+def test_make_peer_checks_its_table():
+    with pytest.raises(ValueError):
+        binding.make_peer(2, 2, [FAKE, FAKE])
+    with pytest.raises(ValueError):
+        binding.make_peer(0, 2, [FAKE])
+    p = binding.make_peer(1, 2, [FAKE, FAKE * 2], [FAKE * 3, FAKE * 4], 7)
+    assert (p.rank, p.world, p.epoch) == (1, 2, 7) and p.recv[1] == FAKE * 2 and p.flags[0] == FAKE * 3

@@ -6,10 +6,12 @@ and runs the stage calls through the fp64 stand-in in tests/tp_cpu_ops.py;
 the collectives are torch.distributed's.  Every rank checks its results
 against the oracle's unsharded block: Y and dX (all-reduced, or its token
 rows in the sequence-parallel form), its shard of dA, da and dB, and db.
-This pins the host logic: which rank adds b, which outputs are reduced,
-gathered or scattered, and the shard and token bounds.  The GEMMs are
-checked on the GPU elsewhere; runs on several GPUs are not possible on a
-one-GPU machine.
+This pins the host logic of the NCCL form (fp32 partials summed by the
+collective, b added once after the sum, which outputs are reduced, gathered
+or scattered, the shard and token bounds) and, with a stand-in for CUDA IPC,
+the peer-table exchange of the fused form.  The GEMMs and the fused
+reduction are checked on the GPU elsewhere; runs on several GPUs are not
+possible on a one-GPU machine.
 """
 import datetime
 import os
@@ -49,8 +51,8 @@ def _worker(rank, world, port, shape, sp, mode, results):
         rows = tp.token_rows(T, rank, world) if sp else slice(0, T)
         X = d["X"][rows] if sp else d["X"]
         dY = d["dY"][rows] if sp else d["dY"]
-        Y, saved = tp.forward(X, A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode, ops=tp_cpu_ops)
-        g = tp.backward(dY, saved, A_i, B_i, sequence_parallel=sp, mode=mode, ops=tp_cpu_ops)
+        Y, saved = tp.forward(X, A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode, reduction="nccl", ops=tp_cpu_ops)
+        g = tp.backward(dY, saved, A_i, B_i, sequence_parallel=sp, mode=mode, reduction="nccl", ops=tp_cpu_ops)
         err = {
             "Y": np.abs(Y.numpy() - ref["Y"][rows]).max(),
             "dX": np.abs(g["dX"].numpy() - ref["dX"][rows]).max(),
@@ -111,3 +113,75 @@ def test_shard_and_token_bounds():
     A1, a1, B1 = tp.shard_parameters(A, a, B, 1, 2)
     assert torch.equal(A1, A[:, 4:]) and torch.equal(a1, a[4:]) and torch.equal(B1, B[4:, :])
     assert A1.is_contiguous() and B1.is_contiguous()
+
+
+# ------------------------------------------------------------------ peer table of the fused form
+class _FakeIpc:
+    """Stand-in for the library's CUDA IPC calls: an address exported by rank
+    r maps, in rank q's process, to 1e12·(q+1) + address (a fake mapping)."""
+    def __init__(self, rank):
+        self.rank = rank
+        self.closed = []
+
+    def mlp_tp_ipc_export(self, ptr):
+        return (f"handle-of-rank-{self.rank}".encode(), ptr % 4096)
+
+    def mlp_tp_ipc_import(self, handle, offset):
+        src = int(handle.decode().rsplit("-", 1)[1])
+        return (self.rank + 1) * 10 ** 12 + src * 10 ** 9 + offset
+
+    def mlp_tp_ipc_close(self, ptr, offset):
+        self.closed.append((ptr, offset))
+
+    def peer_recv_bytes(self, T, h, world):
+        return T * h * 4
+
+    def peer_flag_bytes(self, T, h, world):
+        return 256
+
+    def make_peer(self, rank, world, recv, flags=None, epoch=0):
+        return {"rank": rank, "world": world, "recv": list(recv), "flags": list(flags), "epoch": epoch}
+
+
+def _exchange_worker(rank, world, port, results):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ipc = _FakeIpc(rank)
+        ex = tp.PeerExchange(64 * world, 128, device="cpu", ops=ipc)
+        own = ex.buf.data_ptr()
+        q1, q2 = ex.next(), ex.next()
+        ex.close()
+        results[rank] = {"own": own, "table": ex.table, "q1": q1, "q2": q2, "closed": ipc.closed,
+                         "recv_bytes": ex.recv_bytes}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_exchange_maps_every_other_rank_and_keeps_its_own_pointer():
+    world = 2
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    results = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, world, port, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for rank in range(world):
+        res = results[rank]
+        table = res["table"]
+        assert len(table) == world and table[rank] == res["own"]
+        for src in range(world):
+            if src != rank:
+                # the mapping of rank src's exported buffer, at its offset inside its allocation
+                off = results[src]["own"] % 4096
+                assert table[src] == (rank + 1) * 10 ** 12 + src * 10 ** 9 + off
+        q1, q2 = res["q1"], res["q2"]
+        assert (q1["rank"], q1["world"], q1["epoch"], q2["epoch"]) == (rank, world, 1, 2)
+        assert q1["recv"] == table and q1["flags"] == [a + res["recv_bytes"] for a in table]
+        assert sorted(res["closed"]) == sorted((table[s], results[s]["own"] % 4096) for s in range(world) if s != rank)

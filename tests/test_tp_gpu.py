@@ -2,8 +2,10 @@
 GPU through the C-ABI, as one NCCL rank in a child process.
 
 With one rank the collectives move nothing, but every stage runs through the
-library with the shard shapes the orchestration passes (t = 1 per rank), and
-the results must meet the parity bar against the oracle's unsharded block.
+library with the shard shapes the orchestration passes (t = 1 per rank), in
+both reduction forms (the fused peer-store reduction and the NCCL one over
+fp32 partials), and the results must meet the parity bar against the
+oracle's unsharded block.
 Several ranks need several GPUs; this machine gives one.
 """
 import datetime
@@ -24,7 +26,7 @@ def _free_port():
     return port
 
 
-def _worker(port, sp, mode, results):
+def _worker(port, sp, mode, reduction, results):
     import torch
     import torch.distributed as dist
     from oracle import mlp_oracle as oracle
@@ -41,8 +43,8 @@ def _worker(port, sp, mode, results):
         ref = oracle.full(inp)
         d = {k: v.cuda() for k, v in inp.items()}
         A_i, a_i, B_i = tp.shard_parameters(d["A"], d["a"], d["B"], 0, 1)
-        Y, saved = tp.forward(d["X"], A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode)
-        g = tp.backward(d["dY"], saved, A_i, B_i, sequence_parallel=sp, mode=mode)
+        Y, saved = tp.forward(d["X"], A_i, a_i, B_i, d["b"], sequence_parallel=sp, mode=mode, reduction=reduction)
+        g = tp.backward(d["dY"], saved, A_i, B_i, sequence_parallel=sp, mode=mode, reduction=reduction)
         torch.cuda.synchronize()
         out = dict(g, Y=Y)
         results["ratios"] = {k: worst_ratio(out[k], ref[k]) for k in ("Y", "dX", "dA", "da", "dB", "db")}
@@ -52,11 +54,12 @@ def _worker(port, sp, mode, results):
 
 @pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
 @pytest.mark.parametrize("mode", [0, 3], ids=["accurate", "fast"])
-def test_one_rank_through_the_library_meets_the_bar(sp, mode):
+@pytest.mark.parametrize("reduction", ["peer", "nccl"])
+def test_one_rank_through_the_library_meets_the_bar(sp, mode, reduction):
     ctx = mp.get_context("spawn")
     manager = ctx.Manager()
     results = manager.dict()
-    p = ctx.Process(target=_worker, args=(_free_port(), sp, mode, results))
+    p = ctx.Process(target=_worker, args=(_free_port(), sp, mode, reduction, results))
     p.start()
     p.join(300)
     assert p.exitcode == 0

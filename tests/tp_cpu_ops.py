@@ -1,6 +1,9 @@
 """Test stand-in for the C-ABI stage calls on the CPU, in fp64, for the
 multi-process tests of the cross-GPU orchestration in
 tensor_transformer_mlp_bias_b200.tp.  Same call signatures as the binding.
+The partial-sum calls (the *_peer GEMMs and mlp_tp_peer_reduce) support the
+one-rank view the NCCL form uses: the whole partial written to slot 0 of the
+caller's own buffer, which the descriptor here holds as a tensor.
 
 It computes each stage from the oracle's definitions (GeLU and its derivative
 from oracle/mlp_oracle.py, plain matrix products), writing into the output
@@ -64,3 +67,29 @@ def mlp_tp_fc1_backward_data(dH, dH_lo, A, T, h, f, t, dX, ws, stream=None):
 def mlp_tp_fc1_backward_weight(X, dH, dH_lo, T, h, f, t, dA, ws, stream=None):
     dh = _np(dH) + (_np(dH_lo) if dH_lo is not None else 0.0)
     dA.copy_(torch.from_numpy(np.asarray(_np(X)).T @ dh))
+
+
+class _Peer:
+    def __init__(self, rank, world, recv, flags=None, epoch=0):
+        if world != 1 or epoch != 0:
+            raise NotImplementedError("the CPU stand-in has no cross-process buffers")
+        self.rank, self.world, self.recv, self.epoch = rank, world, list(recv), epoch
+
+
+def make_peer(rank, world, recv, flags=None, epoch=0):
+    return _Peer(rank, world, recv, flags, epoch)
+
+
+def mlp_tp_fc2_forward_peer(H, H_lo, B, T, h, fs, peer, ws, stream=None):
+    hh = _np(H) + (_np(H_lo) if H_lo is not None else 0.0)
+    peer.recv[0].copy_(torch.from_numpy(hh @ _np(B)))
+
+
+def mlp_tp_fc1_backward_data_peer(dH, dH_lo, A, T, h, fs, peer, ws, stream=None):
+    dh = _np(dH) + (_np(dH_lo) if dH_lo is not None else 0.0)
+    peer.recv[0].copy_(torch.from_numpy(dh @ _np(A).T))
+
+
+def mlp_tp_peer_reduce(peer, bias, T, h, out, ws, stream=None):
+    s = _np(peer.recv[0])[:T]
+    out.copy_(torch.from_numpy(s + (_np(bias) if bias is not None else 0.0)))
