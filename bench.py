@@ -344,6 +344,9 @@ def main():
     ap.add_argument("--no-recompute", action="store_true", help="skip the activation-recomputation leg")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     ap.add_argument("--no-steady", action="store_true", help="skip the two-second steady-state leg")
+    ap.add_argument("--no-peer", action="store_true", help="skip the one-GPU leg of the cross-GPU reduction path")
+    ap.add_argument("--stage-steps", type=int, default=None,
+                    help="steps of the per-stage timing pass (default: enough for 0.3 s; small for ncu captures)")
     ap.add_argument("--no-accurate-leg", action="store_true",
                     help="with the fast mode timed, skip timing the accurate mode beside it")
     ap.add_argument("--clock-interval-ms", type=int, default=50,
@@ -434,7 +437,7 @@ def main():
     local_ms = start.elapsed_time(end)
     # per-stage times (events between the stage calls), with the clocks of
     # this window: the roofline's peak follows them
-    n_ev = max(10, args.steps // 4, int(0.3e3 / max(local_ms / args.steps, 1e-3)) + 1)
+    n_ev = args.stage_steps or max(10, args.steps // 4, int(0.3e3 / max(local_ms / args.steps, 1e-3)) + 1)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(n_ev)]
     torch.cuda.synchronize()
     with ClockSampler(local, args.clock_interval_ms) as clk_stages:
@@ -484,6 +487,43 @@ def main():
         steady = {"value": fl_s / (ms_s * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_s / n_s, "steps": n_s,
                   "seconds": ms_s * 1e-3, "clocks": clk_s,
                   "ms_x_mhz": (ms_s / n_s) * clk_s["sm_mhz"] if clk_s.get("sm_mhz") else None}
+
+    # ------------------------------------------------ the cross-GPU reduction path on this one GPU
+    # The row-parallel forward as one rank of a one-rank group: the GEMM whose
+    # epilogue stores the fp32 partial into the (here local) receive buffer and
+    # raises the arrival counts, then the owner's reduce (sum, b, one
+    # rounding).  Same FLOPs as the fc2_forward stage; the reduce kernel is
+    # HBM-bound: 4·T·h bytes read, 2·T·h written.
+    peer = None
+    if not args.no_peer and world == 1 and T % 128 == 0:
+        peer_hbm = None
+        recv = torch.zeros(binding.peer_recv_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
+        flags = torch.zeros(binding.peer_flag_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
+        ws_p = binding.make_workspace(T, h, f, 1)
+        Yp = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+        n_p = max(10, args.steps)
+        evp = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_p + 3)]
+        for k in range(n_p + 3):
+            q = binding.make_peer(0, 1, [recv], [flags], k + 1)
+            evp[k][0].record(stream)
+            binding.mlp_tp_fc2_forward_peer(H, H_lo2, dev["B"], T, h, f, q, ws_p, sh)
+            evp[k][1].record(stream)
+            binding.mlp_tp_peer_reduce(q, dev["b"], T, h, Yp, ws_p, sh)
+            evp[k][2].record(stream)
+        torch.cuda.synchronize()
+        binding.mlp_tp_check(ws_p, sh)
+        g_ms = statistics.mean(evp[k][0].elapsed_time(evp[k][1]) for k in range(3, n_p + 3))
+        r_ms = statistics.mean(evp[k][1].elapsed_time(evp[k][2]) for k in range(3, n_p + 3))
+        rbytes = 4.0 * T * h + 2.0 * T * h + 2.0 * h
+        peaks_p, _ = load_peaks()
+        peer_hbm = float(peaks_p.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        peer = {"gemm_ms": g_ms, "gemm_tflops": 2.0 * T * h * f * (1 if mode & 1 else 2) / (g_ms * 1e-3) / 1e12,
+                "reduce_ms": r_ms, "reduce_gbs": rbytes / (r_ms * 1e-3) / 1e9,
+                "reduce_frac_of_hbm": rbytes / (r_ms * 1e-3) / 1e9 / peer_hbm, "hbm_peak_gbs": peer_hbm,
+                "reduce_bytes": rbytes, "steps": n_p,
+                "api": "mlp_tp_fc2_forward_peer + mlp_tp_peer_reduce, one rank (world = 1), flags on; "
+                       "gemm_tflops counts the tensor products the GEMM runs"}
+        del recv, flags, ws_p
 
     # ------------------------------------------------ the workload's other shard counts
     # Same device-resident step (stage calls) for every other t the workload
@@ -718,6 +758,8 @@ def main():
         line["accurate"] = accurate
     if steady is not None:
         line["steady"] = steady
+    if peer is not None:
+        line["peer"] = peer
     if graph is not None:
         line["graph"] = graph
     if recompute is not None:
