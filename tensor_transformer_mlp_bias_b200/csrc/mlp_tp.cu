@@ -595,7 +595,10 @@ mlp_status_t fc1_forward(const Shape& s, const void* X, const void* A, const voi
       const int64_t waves = (tiles + pairs - 1) / pairs;
       return static_cast<double>(tiles) / static_cast<double>(waves * pairs);
     };
-    if (wave_eff(512) + 0.05 >= wave_eff(256))
+    // When even the 256-column tiles fit in one wave, they win outright: twice
+    // the CTA pairs, each with half the (here unhidden) epilogue.
+    const int64_t tiles256 = mt * ((s.f + 255) / 256);
+    if (tiles256 > pairs && wave_eff(512) + 0.05 >= wave_eff(256))
       return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H)");
   }
   return launch_gemm<false, true, EPI_BIAS_GELU, 256>(g, p, L, "column-parallel forward (Z, H)");

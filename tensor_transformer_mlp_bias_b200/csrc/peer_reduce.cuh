@@ -11,6 +11,8 @@
 
 namespace mlptp {
 
+constexpr int PEER_ROWS_IN_FLIGHT = 8;  // rows of loads each thread keeps in flight
+
 // The owner's side: one CTA of 256 threads per (128-row block, 256-column
 // block) of this rank's token rows.  Thread x of 64 owns 4 consecutive
 // columns; the 4 row phases walk the block's rows.
@@ -48,25 +50,45 @@ __global__ void __launch_bounds__(256) peer_reduce_kernel(const PeerParams q, co
       b[3] = __high2float(b23);
     }
     const size_t slot = static_cast<size_t>(q.rows) * static_cast<size_t>(N);
-    for (int r = static_cast<int>(threadIdx.x) >> 6; r < PEER_BLOCK_ROWS; r += 4) {
-      const int lr = lb * PEER_BLOCK_ROWS + r;
-      if (lr >= q.rows) break;
-      const size_t off = static_cast<size_t>(lr) * static_cast<size_t>(N) + col;
-      if (!index_ok(static_cast<long long>((q.world - 1) * slot + off + 3), recv_elems, status, 0x50au)) break;
-      float4 acc = __ldcg(reinterpret_cast<const float4*>(recv + off));
-      for (int s = 1; s < q.world; ++s) {  // rank order
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(recv + s * slot + off));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    // PEER_ROWS_IN_FLIGHT rows per thread per pass (4 row phases), every
+    // slot's loads issued before the sums use them
+    constexpr int RIF = PEER_ROWS_IN_FLIGHT;
+    for (int r0 = static_cast<int>(threadIdx.x) >> 6; r0 < PEER_BLOCK_ROWS; r0 += 4 * RIF) {
+      float4 acc[RIF];
+      size_t off[RIF];
+      bool live[RIF];
+#pragma unroll
+      for (int j = 0; j < RIF; ++j) {
+        const int lr = lb * PEER_BLOCK_ROWS + r0 + 4 * j;
+        off[j] = static_cast<size_t>(lr) * static_cast<size_t>(N) + col;
+        live[j] = r0 + 4 * j < PEER_BLOCK_ROWS && lr < q.rows &&
+                  index_ok(static_cast<long long>((q.world - 1) * slot + off[j] + 3), recv_elems, status, 0x50au);
+        acc[j] = live[j] ? __ldcg(reinterpret_cast<const float4*>(recv + off[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x + b[0], acc.y + b[1]);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z + b[2], acc.w + b[3]);
-      uint2 o;
-      o.x = *reinterpret_cast<uint32_t*>(&lo);
-      o.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(out + off) = o;
+      for (int s = 1; s < q.world; ++s) {  // rank order
+        float4 v[RIF];
+#pragma unroll
+        for (int j = 0; j < RIF; ++j)
+          v[j] = live[j] ? __ldcg(reinterpret_cast<const float4*>(recv + s * slot + off[j]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < RIF; ++j) {
+          acc[j].x += v[j].x;
+          acc[j].y += v[j].y;
+          acc[j].z += v[j].z;
+          acc[j].w += v[j].w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < RIF; ++j) {
+        if (!live[j]) continue;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x + b[0], acc[j].y + b[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z + b[2], acc[j].w + b[3]);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t*>(&lo);
+        o.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out + off[j]) = o;
+      }
     }
   }
   if (q.epoch != 0u) {
