@@ -807,9 +807,12 @@ def traffic_for(stage, wl, t):
 
 
 def kernel_source_digest():
+    """First 12 hex digits of the sha256 of the sources that make the GEMM
+    kernels and their launch shapes (the kernels whose DRAM traffic the
+    roofline reports)."""
     import hashlib
     hsh = hashlib.sha256()
-    for n in ("gemm.cuh", "ptx.cuh", "colsum.cuh", "peer.cuh", "peer_reduce.cuh", "mlp_tp.cu"):
+    for n in ("gemm.cuh", "ptx.cuh", "peer.cuh", "mlp_tp.cu"):
         with open(os.path.join(ROOT, "tensor_transformer_mlp_bias_b200", "csrc", n), "rb") as fh:
             hsh.update(fh.read())
     return hsh.hexdigest()[:12]

@@ -11,12 +11,12 @@
 
 namespace mlptp {
 
-constexpr int PEER_ROWS_IN_FLIGHT = 8;  // rows of loads each thread keeps in flight
+constexpr int PEER_ROWS_IN_FLIGHT = 4;  // rows of loads each thread keeps in flight
 
 // The owner's side: one CTA of 256 threads per (128-row block, 256-column
 // block) of this rank's token rows.  Thread x of 64 owns 4 consecutive
 // columns; the 4 row phases walk the block's rows.
-__global__ void __launch_bounds__(256) peer_reduce_kernel(const PeerParams q, const __nv_bfloat16* __restrict__ bias,
+__global__ void __launch_bounds__(256, 4) peer_reduce_kernel(const PeerParams q, const __nv_bfloat16* __restrict__ bias,
                                                           int N, __nv_bfloat16* __restrict__ out, unsigned int* status,
                                                           unsigned long long budget_ns, long long recv_elems) {
   const int lb = static_cast<int>(blockIdx.x) / q.ncb;
@@ -51,26 +51,28 @@ __global__ void __launch_bounds__(256) peer_reduce_kernel(const PeerParams q, co
     }
     const size_t slot = static_cast<size_t>(q.rows) * static_cast<size_t>(N);
     // PEER_ROWS_IN_FLIGHT rows per thread per pass (4 row phases), every
-    // slot's loads issued before the sums use them
+    // slot's loads issued before the sums use them; few enough registers that
+    // the grid (one CTA per block) fits one wave
     constexpr int RIF = PEER_ROWS_IN_FLIGHT;
-    for (int r0 = static_cast<int>(threadIdx.x) >> 6; r0 < PEER_BLOCK_ROWS; r0 += 4 * RIF) {
+    const int rows_here = min(PEER_BLOCK_ROWS, q.rows - lb * PEER_BLOCK_ROWS);
+    const size_t step = static_cast<size_t>(4) * static_cast<size_t>(N);
+    for (int r0 = static_cast<int>(threadIdx.x) >> 6; r0 < rows_here; r0 += 4 * RIF) {
+      const size_t off0 = static_cast<size_t>(lb * PEER_BLOCK_ROWS + r0) * static_cast<size_t>(N) + col;
+      const int live = min(RIF, (rows_here - r0 + 3) / 4);  // rows r0, r0+4, ... below rows_here
+      if (!index_ok(static_cast<long long>((q.world - 1) * slot + off0 + (live - 1) * step + 3), recv_elems, status,
+                    0x50au))
+        break;
       float4 acc[RIF];
-      size_t off[RIF];
-      bool live[RIF];
 #pragma unroll
-      for (int j = 0; j < RIF; ++j) {
-        const int lr = lb * PEER_BLOCK_ROWS + r0 + 4 * j;
-        off[j] = static_cast<size_t>(lr) * static_cast<size_t>(N) + col;
-        live[j] = r0 + 4 * j < PEER_BLOCK_ROWS && lr < q.rows &&
-                  index_ok(static_cast<long long>((q.world - 1) * slot + off[j] + 3), recv_elems, status, 0x50au);
-        acc[j] = live[j] ? __ldcg(reinterpret_cast<const float4*>(recv + off[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int j = 0; j < RIF; ++j)
+        acc[j] = j < live ? __ldcg(reinterpret_cast<const float4*>(recv + off0 + j * step)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
       for (int s = 1; s < q.world; ++s) {  // rank order
+        const float* src = recv + s * slot + off0;
         float4 v[RIF];
 #pragma unroll
         for (int j = 0; j < RIF; ++j)
-          v[j] = live[j] ? __ldcg(reinterpret_cast<const float4*>(recv + s * slot + off[j]))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[j] = j < live ? __ldcg(reinterpret_cast<const float4*>(src + j * step)) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < RIF; ++j) {
           acc[j].x += v[j].x;
@@ -81,13 +83,13 @@ __global__ void __launch_bounds__(256) peer_reduce_kernel(const PeerParams q, co
       }
 #pragma unroll
       for (int j = 0; j < RIF; ++j) {
-        if (!live[j]) continue;
+        if (j >= live) continue;
         __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x + b[0], acc[j].y + b[1]);
         __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z + b[2], acc[j].w + b[3]);
         uint2 o;
         o.x = *reinterpret_cast<uint32_t*>(&lo);
         o.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(out + off[j]) = o;
+        *reinterpret_cast<uint2*>(out + off0 + j * step) = o;
       }
     }
   }
