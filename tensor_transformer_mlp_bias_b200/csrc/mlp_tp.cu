@@ -254,10 +254,49 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps, cached per host thread.  A map holds only the base
+// address, the extents, the row stride, the box and the element format and
+// swizzle, so an entry whose key matches all of those is the map the driver
+// would encode again; a launch-bound step (small batches) spends much of its
+// host time encoding about seven maps per GEMM otherwise.
+struct MapKey {
+  const void* ptr;
+  int64_t rows, cols;
+  uint32_t box0, box1;
+  int kind;  // 0: bf16 operand (128-byte swizzle), 1: bf16 output (64-byte), 2: fp32 output (128-byte)
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && box0 == o.box0 && box1 == o.box1 && kind == o.kind;
+  }
+};
+struct MapCache {
+  static constexpr int N = 64;
+  MapKey key[N];
+  CUtensorMap map[N];
+  bool used[N] = {};
+  int next = 0;
+  bool find(const MapKey& k, CUtensorMap* out) const {
+    for (int i = 0; i < N; ++i)
+      if (used[i] && key[i] == k) {
+        *out = map[i];
+        return true;
+      }
+    return false;
+  }
+  void put(const MapKey& k, const CUtensorMap& m) {
+    key[next] = k;
+    map[next] = m;
+    used[next] = true;
+    next = (next + 1) % N;
+  }
+};
+thread_local MapCache g_map_cache;
+
 // 2-D bf16 row-major matrix [rows, cols] (cols contiguous), box of
 // 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
 mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, uint32_t box_rows,
                       const char* name) {
+  const MapKey key{ptr, rows, cols, 64u, box_rows, 0};
+  if (g_map_cache.find(key, map)) return MLP_OK;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -268,6 +307,7 @@ mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t c
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for %s (CUresult %d)", name, (int)r);
+  g_map_cache.put(key, *map);
   return MLP_OK;
 }
 
@@ -275,6 +315,8 @@ mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t c
 // from the epilogue's swizzled staging tiles (bf16: 64-byte swizzle, fp32:
 // 128-byte swizzle, matching the staging layout in gemm.cuh).
 mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, bool f32, const char* name) {
+  const MapKey key{ptr, rows, cols, 32u, 32u, f32 ? 2 : 1};
+  if (g_map_cache.find(key, map)) return MLP_OK;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t esz = f32 ? 4 : 2;
@@ -288,6 +330,7 @@ mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for output of %s (CUresult %d)", name, (int)r);
+  g_map_cache.put(key, *map);
   return MLP_OK;
 }
 
