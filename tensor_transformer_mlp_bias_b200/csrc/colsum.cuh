@@ -30,6 +30,10 @@ constexpr int COLSUM_PHASES = 32;  // row phases per block in pass 1
 __global__ void __launch_bounds__(32 * COLSUM_PHASES) colsum_partial(const __nv_bfloat16* __restrict__ m, int R,
                                                                      int C, float* __restrict__ partial,
                                                                      long long partial_elems, unsigned int* status) {
+  // launched with programmatic dependent launch: every global access below
+  // follows the previous grid's completion
+  grid_wait_prerequisites();
+  grid_launch_dependents();
   __shared__ float red[COLSUM_PHASES][32][9];
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int c0 = (blockIdx.x * 32 + tx) * 8;
@@ -77,6 +81,8 @@ __global__ void __launch_bounds__(32 * COLSUM_PHASES) colsum_partial(const __nv_
 __global__ void __launch_bounds__(256) colsum_final(const float* __restrict__ partial, int chunks, int C,
                                                     __nv_bfloat16* __restrict__ out, long long partial_elems,
                                                     unsigned int* status) {
+  grid_wait_prerequisites();
+  grid_launch_dependents();
   __shared__ float red[8][33];
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int c = blockIdx.x * 32 + tx;

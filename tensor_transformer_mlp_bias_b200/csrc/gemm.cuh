@@ -921,6 +921,8 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
 // columns of one row of one split tile.
 template <int TILE_M, int TILE_N>
 __global__ void __launch_bounds__(256) split_reduce_kernel(const GemmParams p, int first_tile, int tiles, int split) {
+  grid_wait_prerequisites();  // programmatic dependent launch, as the GEMMs
+  grid_launch_dependents();
   constexpr int COLS8 = TILE_N / 8;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(tiles) * TILE_M * COLS8) return;

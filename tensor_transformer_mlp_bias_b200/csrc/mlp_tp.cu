@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/mlp_tp.h"
 #include "colsum.cuh"
@@ -414,6 +415,26 @@ struct Launch {
   cudaStream_t stream;
 };
 
+// Launches a helper kernel (column sums, split-tile reduce, peer reduce)
+// with programmatic dependent launch, as the GEMMs: it may be scheduled while
+// the previous kernel drains, and waits for it (griddepcontrol.wait) before
+// its first global access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_helper(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8, bool DUAL = false>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
   using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
@@ -540,9 +561,8 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
     const int tiles = p.num_tiles - first;
     const int split = p.kb_split > 1 ? p.kb_split : p.tail_split;
     const long long threads = static_cast<long long>(tiles) * Cfg::TILE_M * (Cfg::TILE_N / 8);
-    split_reduce_kernel<Cfg::TILE_M, Cfg::TILE_N>
-        <<<static_cast<unsigned>((threads + 255) / 256), 256, 0, L.stream>>>(p, first, tiles, split);
-    e = cudaGetLastError();
+    e = launch_helper(split_reduce_kernel<Cfg::TILE_M, Cfg::TILE_N>, dim3(static_cast<unsigned>((threads + 255) / 256)),
+                      dim3(256), L.stream, p, first, tiles, split);
     if (e != cudaSuccess) return cuda_fail(e, "split_reduce");
     g_launches.fetch_add(1);
   }
@@ -553,10 +573,9 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
 // workspace status word (NULL: none); both serve the bounds-checking build.
 mlp_status_t launch_colsum_final(const float* partial, int chunks, int64_t C, void* out, cudaStream_t stream,
                                  size_t partial_elems, unsigned int* status) {
-  colsum_final<<<static_cast<unsigned>((C + 31) / 32), dim3(32, 8), 0, stream>>>(
-      partial, chunks, static_cast<int>(C), static_cast<__nv_bfloat16*>(out), static_cast<long long>(partial_elems),
-      status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_helper(colsum_final, dim3(static_cast<unsigned>((C + 31) / 32)), dim3(32, 8), stream, partial,
+                                chunks, static_cast<int>(C), static_cast<__nv_bfloat16*>(out),
+                                static_cast<long long>(partial_elems), status);
   if (e != cudaSuccess) return cuda_fail(e, "colsum_final");
   g_launches.fetch_add(1);
   return MLP_OK;
@@ -570,10 +589,9 @@ mlp_status_t launch_colsum(const void* m, int64_t R, int64_t C, void* out, float
   }
   const int chunks = static_cast<int>(colsum_chunks(R));
   dim3 grid1(static_cast<unsigned>((C + COLSUM_COLS_PER_BLOCK - 1) / COLSUM_COLS_PER_BLOCK), chunks);
-  colsum_partial<<<grid1, dim3(32, COLSUM_PHASES), 0, stream>>>(static_cast<const __nv_bfloat16*>(m), static_cast<int>(R),
-                                                    static_cast<int>(C), partial,
-                                                    static_cast<long long>(partial_elems), status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_helper(colsum_partial, grid1, dim3(32, COLSUM_PHASES), stream,
+                                static_cast<const __nv_bfloat16*>(m), static_cast<int>(R), static_cast<int>(C), partial,
+                                static_cast<long long>(partial_elems), status);
   if (e != cudaSuccess) return cuda_fail(e, "colsum_partial");
   g_launches.fetch_add(1);
   return launch_colsum_final(partial, chunks, C, out, stream, partial_elems, status);
@@ -1072,10 +1090,10 @@ mlp_status_t mlp_tp_peer_reduce(const mlp_tp_peer_t* peer, const void* bias, int
   if ((st = current_device(dev, sms)) != MLP_OK) return st;
   const long long blocks = static_cast<long long>(q.nbl) * q.ncb;
   if (blocks == 0) return MLP_OK;
-  peer_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      q, static_cast<const __nv_bfloat16*>(bias), static_cast<int>(h), static_cast<__nv_bfloat16*>(out),
-      static_cast<unsigned int*>(ws), g_budget_ns.load(), recv_elems);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_helper(peer_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                                static_cast<cudaStream_t>(stream), q, static_cast<const __nv_bfloat16*>(bias),
+                                static_cast<int>(h), static_cast<__nv_bfloat16*>(out), static_cast<unsigned int*>(ws),
+                                static_cast<unsigned long long>(g_budget_ns.load()), recv_elems);
   if (e != cudaSuccess) return cuda_fail(e, "peer_reduce");
   g_launches.fetch_add(1);
   return MLP_OK;

@@ -19,6 +19,8 @@ constexpr int PEER_ROWS_IN_FLIGHT = 4;  // rows of loads each thread keeps in fl
 __global__ void __launch_bounds__(256, 4) peer_reduce_kernel(const PeerParams q, const __nv_bfloat16* __restrict__ bias,
                                                           int N, __nv_bfloat16* __restrict__ out, unsigned int* status,
                                                           unsigned long long budget_ns, long long recv_elems) {
+  grid_wait_prerequisites();  // programmatic dependent launch, as the GEMMs
+  grid_launch_dependents();
   const int lb = static_cast<int>(blockIdx.x) / q.ncb;
   const int cb = static_cast<int>(blockIdx.x) % q.ncb;
   __shared__ int go;
