@@ -495,7 +495,7 @@ def main():
     # rounding).  Same FLOPs as the fc2_forward stage; the reduce kernel is
     # HBM-bound: 4·T·h bytes read, 2·T·h written.
     peer = None
-    if not args.no_peer and world == 1 and T % 128 == 0:
+    if not args.no_peer and world == 1:
         peer_hbm = None
         recv = torch.zeros(binding.peer_recv_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
         flags = torch.zeros(binding.peer_flag_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
