@@ -758,6 +758,7 @@ mlp_status_t check_peer(const mlp_tp_peer_t* peer, int64_t T, int64_t h, PeerPar
   if (world < 1 || world > MLP_TP_MAX_WORLD)
     return fail(MLP_ERR_INVALID_ARG, "peer world %d outside 1..%d", world, MLP_TP_MAX_WORLD);
   if (rank < 0 || rank >= world) return fail(MLP_ERR_INVALID_ARG, "peer rank %d outside 0..%d", rank, world - 1);
+  if (peer->reserved != 0u) return fail(MLP_ERR_INVALID_ARG, "peer descriptor's reserved field is not 0");
   if (T % world != 0)
     return fail(MLP_ERR_UNSUPPORTED_SHAPE, "T=%lld tokens do not split over %d ranks", (long long)T, world);
   const PeerShape ps = peer_shape(T, h, world);

@@ -112,6 +112,7 @@ class Saved:
     H_lo: torch.Tensor
     ws: object           # workspace of this rank's stage calls
     exchange: Optional[PeerExchange] = None
+    owns_exchange: bool = False  # created by forward(): the backward closes it
 
 
 def shard_bounds(f: int, rank: int, world: int) -> Tuple[int, int]:
@@ -192,7 +193,8 @@ def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Te
     fs = A_i.shape[1]
     dt, zdt = _dtypes(ops)
     dev = X.device
-    if reduction == "peer" and exchange is None:
+    owns = reduction == "peer" and exchange is None
+    if owns:
         exchange = PeerExchange(T, h, group, dev, ops)
     ws = ops.make_workspace(T, h, fs, 1, dev)
     Z = torch.empty(T, fs, dtype=zdt, device=dev)
@@ -203,7 +205,7 @@ def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Te
     Y = _sum_partials(lambda q: ops.mlp_tp_fc2_forward_peer(H, lo, B_i, T, h, fs, q, ws), b, T, h, dev,
                       group=group, sequence_parallel=sequence_parallel, reduction=reduction, exchange=exchange,
                       ws=ws, ops=ops)
-    return Y, Saved(X, Z, H, H_lo, ws, exchange)
+    return Y, Saved(X, Z, H, H_lo, ws, exchange, owns)
 
 
 def backward(dY: torch.Tensor, saved: Saved, A_i: torch.Tensor, B_i: torch.Tensor, *, group=None,
@@ -224,14 +226,21 @@ def backward(dY: torch.Tensor, saved: Saved, A_i: torch.Tensor, B_i: torch.Tenso
     dB, db = e(fs, h), e(h)
     ops.mlp_tp_fc2_backward_weight(saved.H, saved.H_lo, dY, T, h, fs, 1, dB, db, saved.ws)
     lo = None if mode & binding.FAST_FC1_BACKWARD_DATA else dH_lo
-    exchange = saved.exchange
+    exchange, owns = saved.exchange, saved.owns_exchange
     if reduction == "peer" and exchange is None:
-        exchange = PeerExchange(T, h, group, dev, ops)
+        exchange, owns = PeerExchange(T, h, group, dev, ops), True
     dX = _sum_partials(lambda q: ops.mlp_tp_fc1_backward_data_peer(dH, lo, A_i, T, h, fs, q, saved.ws), None,
                        T, h, dev, group=group, sequence_parallel=sequence_parallel, reduction=reduction,
                        exchange=exchange, ws=saved.ws, ops=ops)
     dA = e(h, fs)
     ops.mlp_tp_fc1_backward_weight(saved.X, dH, dH_lo, T, h, fs, 1, dA, saved.ws)
+    if owns:
+        # the exchange's buffers are read by this rank's last reduce and by the
+        # other ranks' GEMMs: every rank syncs and meets before it unmaps
+        if dev.type == "cuda":
+            torch.cuda.synchronize(dev)
+        dist.barrier(group=group)
+        exchange.close()
     return {"dX": dX, "dA": dA, "da": da, "dB": dB, "db": db}
 
 

@@ -198,6 +198,7 @@ def _fc2_peer(lib, peer, T=512, h=256, fs=128):
     (dict(world=2, recv=[FAKE, None]), 1, "receive buffer 1 is NULL"),
     (dict(world=2, recv=[FAKE, FAKE + 4]), 3, "receive buffer 1 is not 16-byte aligned"),
     (dict(world=2, epoch=1, flags=None), 1, "flag block 0 is NULL"),
+    (dict(reserved=5), 1, "reserved"),
 ])
 def test_peer_descriptor_is_validated_on_the_host(lib, kw, status, needle):
     if kw is None:
@@ -208,6 +209,7 @@ def test_peer_descriptor_is_validated_on_the_host(lib, kw, status, needle):
         flags = kw.get("flags", [FAKE] * world)
         peer = binding.Peer()
         peer.rank, peer.world, peer.epoch = kw.get("rank", 0), world, kw.get("epoch", 0)
+        peer.reserved = kw.get("reserved", 0)
         for o in range(min(world, binding.MAX_WORLD)):
             peer.recv[o] = recv[o]
             peer.flags[o] = flags[o] if flags is not None else None
