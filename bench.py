@@ -482,8 +482,27 @@ def main():
     # ------------------------------------------------ steady state: the same loop for >= 2 s
     steady = None
     if not args.no_steady:
-        n_s = max(args.steps, int(STEADY_SECONDS * 1e3 / max(ms_per_step, 1e-3)) + 1)
-        ms_s, fl_s, clk_s = timed_loop(n_s)
+        # blocks of about 0.25 s, each timed by its own events, until their
+        # device time adds up to STEADY_SECONDS (the same count on every rank)
+        block = max(args.steps, int(250.0 / max(ms_per_step, 1e-3)) + 1)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        n_s, ms_s = 0, 0.0
+        with ClockSampler(local, args.clock_interval_ms) as clk_st:
+            while ms_s < STEADY_SECONDS * 1e3:
+                b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                b0.record(stream)
+                for _ in range(block):
+                    step()
+                b1.record(stream)
+                torch.cuda.synchronize()
+                ms_b, _ = reduce_max_sum(b0.elapsed_time(b1), 0.0)
+                ms_s += ms_b
+                n_s += block
+        binding.mlp_tp_check(ws, sh)
+        _, fl_s = reduce_max_sum(0.0, float(wl.flops) * n_s)
+        clk_s = clk_st.summary()
         steady = {"value": fl_s / (ms_s * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_s / n_s, "steps": n_s,
                   "seconds": ms_s * 1e-3, "clocks": clk_s,
                   "ms_x_mhz": (ms_s / n_s) * clk_s["sm_mhz"] if clk_s.get("sm_mhz") else None}
