@@ -77,8 +77,8 @@ def test_one_rank_matches_the_single_gpu_stage_calls(T, h, f):
         assert torch.equal(bits(dX), bits(dX_ref)), e_dx
 
 
-@pytest.mark.parametrize("N,mode", [(2, binding.ACCURATE), (4, binding.ACCURATE), (4, binding.FAST)],
-                         ids=["N2", "N4", "N4_fast"])
+@pytest.mark.parametrize("N,mode", [(2, binding.ACCURATE), (4, binding.ACCURATE), (4, binding.FAST),
+                                    (8, binding.ACCURATE)], ids=["N2", "N4", "N4_fast", "N8"])
 def test_emulated_ranks_sum_to_the_unsharded_block(N, mode):
     T, h, f = 512 * N // 2, 384, 2048  # T/N a multiple of 128; h ends in a ragged 256-column block
     fs = f // N
@@ -200,3 +200,18 @@ def test_shapes_the_token_split_cannot_serve_are_refused(T, world):
     with pytest.raises(binding.MlpError) as e:
         binding.mlp_tp_fc2_forward_peer(H, None, B, T, h, fs, q, ws)
     assert e.value.status == 2
+
+
+def test_empty_token_batch_moves_nothing():
+    """T = 0: the GEMMs launch nothing and the reduce has no block; flags stay as they were."""
+    h, fs = 256, 128
+    for world in (1, 2):
+        recv = _zeros_bytes(max(binding.peer_recv_bytes(0, h, world), 256))
+        flags = _zeros_bytes(max(binding.peer_flag_bytes(0, h, world), 256))
+        q = binding.make_peer(0, world, [recv] * world, [flags] * world, 1)
+        B = torch.zeros(fs, h, dtype=torch.bfloat16, device="cuda")
+        ws = binding.make_workspace(0, h, fs, 1)
+        binding.mlp_tp_fc2_forward_peer(None, None, B, 0, h, fs, q, ws)
+        binding.mlp_tp_peer_reduce(q, None, 0, h, None, ws)
+        binding.mlp_tp_check(ws)
+        assert int(flags.sum()) == 0
