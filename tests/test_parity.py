@@ -280,3 +280,25 @@ def test_large_preactivations_saturate_gelu():
     for k in out:
         assert bool(torch.isfinite(out[k].float()).all()), k
     check_full(out, ref)
+
+
+# ------------------------------------------------------------------ seeded random shapes
+def _random_shapes(n=12, seed=2024):
+    """Ragged token counts, hidden sizes and shard widths (multiples of 64), 1-8 shards, both modes."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        t = int(rng.integers(1, 9))
+        fs = 64 * int(rng.integers(1, 7))
+        h = 64 * int(rng.integers(1, 11))
+        T = int(rng.integers(1, 700))
+        mode = ACCURATE if rng.random() < 0.5 else FAST
+        out.append((T, h, fs * t, t, mode))
+    return out
+
+
+@pytest.mark.parametrize("shape", _random_shapes(), ids=lambda s: "T%d_h%d_f%d_t%d_m%d" % s)
+def test_random_shapes_full_oracle(shape):
+    T, h, f, t, mode = shape
+    inp = inputs.make_custom(T, h, f, seed=T * 7 + h + f + t)
+    check_full(run_all(to_gpu(inp), t, mode), oracle.full(inp))
