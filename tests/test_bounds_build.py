@@ -6,8 +6,9 @@ reduce, the bias-gradient column sums) checks its index against its buffer
 and reports MLP_ERR_BOUNDS from mlp_tp_check instead of touching memory
 outside it.  It stands in for a memory checker, which this machine does not
 offer.  The shapes below reach every checked site: split shard-sum tails,
-K-split weight gradients, ragged tiles, da and db, and a batch whose [T, f]
-tensors hold more than 2^31 elements.  They must pass with a clean status
+K-split weight gradients, ragged tiles, da and db, a batch whose [T, f]
+tensors hold more than 2^31 elements, the allocation-free path, and the
+cross-GPU path's peer stores and reduce (two ranks emulated on this GPU).  They must pass with a clean status
 word and meet the parity bar.
 """
 import os
@@ -63,6 +64,41 @@ db = torch.empty(h, dtype=torch.bfloat16, device="cuda")  # h elements, as the c
 binding.mlp_tp_fc2_bias_grad_noalloc(dY, T, h, db)
 binding.mlp_tp_check(None)  # the allocation-free path's own status word: raises on MLP_ERR_BOUNDS
 assert_close("db (allocation-free)", db, dY.double().sum(0).cpu().numpy())
+# the cross-GPU path: peer stores from the GEMM epilogue and the owner's reduce, two ranks emulated in stream
+# order on this GPU (no wait spins), forward and backward partials on the same buffers
+from tensor_transformer_mlp_bias_b200 import tp
+T, h, f, N = 512, 384, 1024, 2
+host = inputs.make_custom(T, h, f, seed=81)
+inp = to_gpu(host)
+ref = oracle.full(host)
+fs = f // N
+rb, fb = binding.peer_recv_bytes(T, h, N), binding.peer_flag_bytes(T, h, N)
+recv = [torch.zeros(rb, dtype=torch.uint8, device="cuda") for _ in range(N)]
+flags = [torch.zeros(fb, dtype=torch.uint8, device="cuda") for _ in range(N)]
+acts = []
+for r in range(N):
+    A_i, a_i, B_i = tp.shard_parameters(inp["A"], inp["a"], inp["B"], r, N)
+    ws = binding.make_workspace(T, h, fs, 1)
+    Z = torch.empty(T, fs, dtype=torch.float32, device="cuda")
+    H, H_lo, dH, dH_lo = (torch.empty(T, fs, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    binding.mlp_tp_fc1_forward(inp["X"], A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws)
+    binding.mlp_tp_fc2_backward_data(inp["dY"], B_i, Z, T, h, fs, 1, dH, dH_lo, None, ws)
+    acts.append((A_i, B_i, H, H_lo, dH, dH_lo, ws))
+for epoch, what in ((1, "Y"), (2, "dX")):
+    qs = [binding.make_peer(r, N, recv, flags, epoch) for r in range(N)]
+    for r, (A_i, B_i, H, H_lo, dH, dH_lo, ws) in enumerate(acts):
+        if what == "Y":
+            binding.mlp_tp_fc2_forward_peer(H, H_lo, B_i, T, h, fs, qs[r], ws)
+        else:
+            binding.mlp_tp_fc1_backward_data_peer(dH, dH_lo, A_i, T, h, fs, qs[r], ws)
+    outs = []
+    for o in range(N):
+        out = torch.empty(T // N, h, dtype=torch.bfloat16, device="cuda")
+        binding.mlp_tp_peer_reduce(qs[o], inp["b"] if what == "Y" else None, T, h, out, acts[o][6])
+        outs.append(out)
+    for a in acts:
+        binding.mlp_tp_check(a[6])  # raises on MLP_ERR_BOUNDS
+    assert_close(what + " (cross-GPU path)", torch.cat(outs), ref[what])
 print("bounds-checked build: clean")
 """
 
