@@ -106,6 +106,14 @@ def test_gpt2_medium_fast_mode():
     check_full(run_all(to_gpu(inp), 8, FAST), ref)
 
 
+@pytest.mark.parametrize("t", [16, 64])
+def test_gpt2_medium_many_shards(t):
+    """Up to 64 shards of 64 columns (the narrowest a shard may be): every shard's K segment is one K slice
+    and each 256-column tile hands its accumulator to the epilogue t times."""
+    inp, ref = _gpt2_medium()
+    check_full(run_all(to_gpu(inp), t), ref)
+
+
 @functools.lru_cache(maxsize=1)
 def _sampled_reference(name):
     """Inputs, sampled indices and the oracle's exact values there; the ffn
