@@ -83,8 +83,11 @@ typedef enum {
   MLP_ERR_UNSUPPORTED_DEVICE = 5,  /* current device is not sm_100, or none */
   MLP_ERR_CUDA = 6,                /* the CUDA runtime reported an error */
   MLP_ERR_TIMEOUT = 7,             /* a kernel's bounded wait ran out (mlp_tp_check) */
-  MLP_ERR_BOUNDS = 8               /* bounds-checking build only: an index fell outside its
+  MLP_ERR_BOUNDS = 8,              /* bounds-checking build only: an index fell outside its
                                       buffer; the access was skipped (mlp_tp_check) */
+  MLP_ERR_RANGE = 9                /* MLP_TP_FP8 only: a value the mode's formats cannot hold
+                                      (|H| or |dH·sH| >= 2^13, or a weight beyond the fp16
+                                      range); the outputs are not valid (mlp_tp_check) */
 } mlp_status_t;
 
 /* Bytes of workspace needed by every entry point below for this shape
@@ -116,8 +119,35 @@ typedef enum {
   MLP_TP_ACCURATE = 0,
   MLP_TP_FAST_FC2_FORWARD = 1,       /* Y  = Σ_i H_i·B_i + b       (high half only) */
   MLP_TP_FAST_FC1_BACKWARD_DATA = 2, /* dX = Σ_i dH_i·A_iᵀ         (high half only) */
-  MLP_TP_FAST = 3                    /* both */
+  MLP_TP_FAST = 3,                   /* both */
+  MLP_TP_FP8 = 4                     /* fp16 operands with e4m3 residual products, below */
 } mlp_tp_mode_t;
+
+/* MLP_TP_FP8: FP8 tensor-core products ("NVIDIA Megatron-LM：大规模Transformer
+ * 模型分布式训练框架", tech-stack item 混合精度: FP8 training on the newer
+ * tensor cores) where they keep the block inside the parity bar.  Operands
+ * enter 8-bit products only as the residual of a 16-bit one:
+ *  - the forward saves Z (fp32), H as fp16 in `H` and the e4m3 residual
+ *    e4m3((g(Z) − H)·2^7) in `H_lo` (T·f bytes of the caller's buffer);
+ *  - Y = Σ_i H_i·fp16(B_i) + b and dX = Σ_i dH16_i·fp16(A_i)ᵀ / sH, one
+ *    fp16 tensor-core product each (11 significant bits);
+ *  - dH16 = fp16(dH·sH) and dH8 = e4m3((dH·sH − dH16)·2^7);
+ *  - dB = (Hᵀ·dY16 + H_loᵀ·dY8) / sY and dA = (X16ᵀ·dH16 + X8ᵀ·dH8)/(sX·sH),
+ *    where X16 = fp16(X·sX), X8 = e4m3(X·sX·2^-7) and the same for dY: an
+ *    fp16 product plus an e4m3 (kind::f8f6f4) product into one fp32
+ *    accumulator, about 15 significant bits for 1.5 bf16-products of tensor
+ *    time instead of the pair's 2.
+ * sX, sY are the largest powers of two with max|X|·sX, max|dY|·sY <= 2^15;
+ * sH the largest with 1.212·max_t‖dY_t‖·max_k‖B_k‖·sH <= 2^12, which bounds
+ * |dH·sH| (Cauchy–Schwarz, max|g'| < 1.2).  The statistics are reduced on
+ * the device each backward; nothing is read back to the host.  Values the
+ * formats cannot hold (|H| >= 2^13; a weight beyond 65504) are reported as
+ * MLP_ERR_RANGE by mlp_tp_check.  Every output stays within
+ * 1e-2·(|exact| + 1) of the exact block on all five workloads the tests run,
+ * the 8.3B-class one included.  This mode needs
+ * mlp_tp_workspace_bytes_mode(..., MLP_TP_FP8) bytes of workspace (the
+ * copies X16, X8, dY16, dY8 and fp16 B or A: 6·T·h + 2·h·f more bytes). */
+size_t mlp_tp_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode);
 
 /* ---------------------------------------------------------------- forward */
 
@@ -208,6 +238,7 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
  * ordinary workspace plus T·f·8 bytes for Z, H, H_lo).  Same conventions
  * and modes as mlp_tp_forward / mlp_tp_backward. */
 size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
+size_t mlp_tp_recompute_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode);
 
 mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* a,
                                       const void* B, const void* b,
@@ -220,6 +251,52 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
                                        int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
                                        void* dX, void* dA, void* da, void* dB, void* db,
                                        void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------- the fp16 + e4m3 mode by stage */
+
+/* The stages of MLP_TP_FP8 (see the mode's description above), for callers
+ * that interleave other work; mlp_tp_forward / mlp_tp_backward with
+ * MLP_TP_FP8 are exactly these calls in this order.  All of them take a
+ * workspace of mlp_tp_workspace_bytes_mode(..., MLP_TP_FP8) bytes, and the
+ * same workspace from the prepare call on:
+ *   forward:  mlp_tp_fp8_prepare_forward (fp16 copy of B into the workspace),
+ *             mlp_tp_fc1_forward_fp8, mlp_tp_fc2_forward_fp8;
+ *   backward: mlp_tp_fp8_prepare_backward (statistics, scales, the fp16 and
+ *             e4m3 copies of X and dY and the fp16 copy of A), then
+ *             mlp_tp_fc2_backward_data_fp8, mlp_tp_fc2_backward_weight_fp8,
+ *             mlp_tp_fc1_backward_data_fp8, mlp_tp_fc1_backward_weight_fp8.
+ * H and dH are fp16 [T,f]; H_lo and dH_lo hold the e4m3 residuals, T·f
+ * bytes.  A stage given the outputs of another mode's stage computes
+ * garbage: the formats differ. */
+mlp_status_t mlp_tp_fp8_prepare_forward(const void* B, int64_t T, int64_t h, int64_t f, int32_t t,
+                                        void* ws, size_t ws_bytes, void* stream);
+mlp_status_t mlp_tp_fp8_prepare_backward(const void* dY, const void* X, const void* A, const void* B,
+                                         int64_t T, int64_t h, int64_t f, int32_t t,
+                                         void* ws, size_t ws_bytes, void* stream);
+mlp_status_t mlp_tp_fc1_forward_fp8(const void* X, const void* A, const void* a,
+                                    int64_t T, int64_t h, int64_t f, int32_t t,
+                                    void* Z, void* H, void* H_lo,
+                                    void* ws, size_t ws_bytes, void* stream);
+/* `b` may be NULL (no bias). */
+mlp_status_t mlp_tp_fc2_forward_fp8(const void* H, const void* b,
+                                    int64_t T, int64_t h, int64_t f, int32_t t,
+                                    void* Y, void* ws, size_t ws_bytes, void* stream);
+/* `da` may be NULL; da is summed from the fp32 dH before any rounding. */
+mlp_status_t mlp_tp_fc2_backward_data_fp8(const void* dY, const void* B, const void* Z,
+                                          int64_t T, int64_t h, int64_t f, int32_t t,
+                                          void* dH, void* dH_lo, void* da,
+                                          void* ws, size_t ws_bytes, void* stream);
+/* `db` may be NULL; db is summed from the bf16 dY. */
+mlp_status_t mlp_tp_fc2_backward_weight_fp8(const void* H, const void* H_lo, const void* dY,
+                                            int64_t T, int64_t h, int64_t f, int32_t t,
+                                            void* dB, void* db,
+                                            void* ws, size_t ws_bytes, void* stream);
+mlp_status_t mlp_tp_fc1_backward_data_fp8(const void* dH,
+                                          int64_t T, int64_t h, int64_t f, int32_t t,
+                                          void* dX, void* ws, size_t ws_bytes, void* stream);
+mlp_status_t mlp_tp_fc1_backward_weight_fp8(const void* dH, const void* dH_lo,
+                                            int64_t T, int64_t h, int64_t f, int32_t t,
+                                            void* dA, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------- across GPUs */
 

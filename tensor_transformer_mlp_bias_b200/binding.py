@@ -26,6 +26,7 @@ STATUS = {
     6: "MLP_ERR_CUDA",
     7: "MLP_ERR_TIMEOUT",
     8: "MLP_ERR_BOUNDS",
+    9: "MLP_ERR_RANGE",
 }
 
 # name -> argument ctypes, in header order
@@ -60,6 +61,17 @@ _SIGS = {
     "mlp_tp_forward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_backward_recompute": ([_P] * 5 + [_I64, _I64, _I64, _I32, _I32] + [_P] * 5 + [_P, _SZ, _P],
                                   ctypes.c_int),
+    "mlp_tp_workspace_bytes_mode": ([_I64, _I64, _I64, _I32, _I32], _SZ),
+    "mlp_tp_recompute_workspace_bytes_mode": ([_I64, _I64, _I64, _I32, _I32], _SZ),
+    "mlp_tp_fp8_prepare_forward": ([_P] + [_I64, _I64, _I64, _I32] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fp8_prepare_backward": ([_P] * 4 + [_I64, _I64, _I64, _I32] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_forward_fp8": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_forward_fp8": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_data_fp8": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 3 + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_backward_weight_fp8": ([_P] * 3 + [_I64, _I64, _I64, _I32] + [_P] * 2 + [_P, _SZ, _P],
+                                       ctypes.c_int),
+    "mlp_tp_fc1_backward_data_fp8": ([_P] + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_weight_fp8": ([_P] * 2 + [_I64, _I64, _I64, _I32] + [_P] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_peer_recv_bytes": ([_I64, _I64, _I32], _SZ),
     "mlp_tp_peer_flag_bytes": ([_I64, _I64, _I32], _SZ),
     "mlp_tp_fc2_forward_peer": ([_P] * 3 + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
@@ -82,6 +94,7 @@ ACCURATE = 0
 FAST_FC2_FORWARD = 1
 FAST_FC1_BACKWARD_DATA = 2
 FAST = 3
+FP8 = 4  # fp16 operands with e4m3 residual products; H, dH fp16 and H_lo, dH_lo e4m3
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -114,7 +127,9 @@ def exported_symbols():
 
 
 # ------------------------------------------------------------------ marshalling
-def _addr(x, name: str, nullable: bool = False):
+def _addr(x, name: str, nullable: bool = False, fmt: str = None):
+    """Device address of `x`.  `fmt` overrides the expected element type:
+    "f16" (fp16) or "e4m3" (one byte per value: uint8 or float8_e4m3fn)."""
     if x is None:
         if nullable:
             return None
@@ -126,9 +141,14 @@ def _addr(x, name: str, nullable: bool = False):
         raise TypeError(f"{name}: expected a torch.Tensor or an int address")
     if x.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor (got {x.device})")
-    want = torch.float32 if name == "Z" else torch.bfloat16
-    if name != "ws" and x.dtype != want:
-        raise ValueError(f"{name} must be {want} (got {x.dtype})")
+    if fmt == "e4m3":
+        want = (torch.uint8, torch.float8_e4m3fn)
+    elif fmt == "f16":
+        want = (torch.float16,)
+    else:
+        want = (torch.float32,) if name == "Z" else (torch.bfloat16,)
+    if name != "ws" and x.dtype not in want:
+        raise ValueError(f"{name} must be {' or '.join(str(w) for w in want)} (got {x.dtype})")
     if not x.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return x.data_ptr()
@@ -170,11 +190,17 @@ def make_workspace(T: int, h: int, f: int, t: int, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def _h_fmts(mode):
+    """Element types of (H, H_lo) and (dH, dH_lo) in a precision mode."""
+    return ("f16", "e4m3") if mode == FP8 else (None, None)
+
+
 def mlp_tp_forward(X, A, a, B, b, T, h, f, t, mode, Y, Z, H, H_lo, ws, stream=None):
     w, wn = _ws(ws)
+    fh, fl = _h_fmts(mode)
     _check(lib().mlp_tp_forward(_addr(X, "X"), _addr(A, "A"), _addr(a, "a"), _addr(B, "B"), _addr(b, "b"),
-                                T, h, f, t, mode, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H"),
-                                _addr(H_lo, "H_lo"), w, wn, _stream(stream)))
+                                T, h, f, t, mode, _addr(Y, "Y"), _addr(Z, "Z"), _addr(H, "H", fmt=fh),
+                                _addr(H_lo, "H_lo", fmt=fl), w, wn, _stream(stream)))
 
 
 def mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, H_lo, ws, stream=None):
@@ -191,8 +217,10 @@ def mlp_tp_fc2_forward(H, H_lo, B, b, T, h, f, t, Y, ws, stream=None):
 
 def mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, mode, dX, dA, da, dB, db, ws, stream=None):
     w, wn = _ws(ws)
+    fh, fl = _h_fmts(mode)
     _check(lib().mlp_tp_backward(_addr(dY, "dY"), _addr(X, "X"), _addr(A, "A"), _addr(B, "B"), _addr(Z, "Z"),
-                                 _addr(H, "H"), _addr(H_lo, "H_lo"), T, h, f, t, mode, _addr(dX, "dX"),
+                                 _addr(H, "H", fmt=fh), _addr(H_lo, "H_lo", fmt=fl), T, h, f, t, mode,
+                                 _addr(dX, "dX"),
                                  _addr(dA, "dA"), _addr(da, "da", True), _addr(dB, "dB"), _addr(db, "db", True),
                                  w, wn, _stream(stream)))
 
@@ -247,6 +275,76 @@ def mlp_tp_backward_recompute(dY, X, A, a, B, T, h, f, t, mode, dX, dA, da, dB, 
                                            _addr(a, "a"), _addr(B, "B"), T, h, f, t, mode,
                                            _addr(dX, "dX", T == 0), _addr(dA, "dA"), _addr(da, "da", True),
                                            _addr(dB, "dB"), _addr(db, "db", True), w, wn, _stream(stream)))
+
+
+def workspace_bytes_mode(T: int, h: int, f: int, t: int, mode: int) -> int:
+    return int(lib().mlp_tp_workspace_bytes_mode(T, h, f, t, mode))
+
+
+def recompute_workspace_bytes_mode(T: int, h: int, f: int, t: int, mode: int) -> int:
+    return int(lib().mlp_tp_recompute_workspace_bytes_mode(T, h, f, t, mode))
+
+
+def make_workspace_mode(T: int, h: int, f: int, t: int, mode: int, recompute: bool = False, device="cuda"):
+    """Zero-filled workspace for a precision mode (MLP_TP_FP8 needs more)."""
+    import torch
+    n = (recompute_workspace_bytes_mode if recompute else workspace_bytes_mode)(T, h, f, t, mode)
+    if n == 0:
+        raise MlpError(2, f"unsupported shape or mode T={T} h={h} f={f} t={t} mode={mode}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ the fp16 + e4m3 mode by stage
+def mlp_tp_fp8_prepare_forward(B, T, h, f, t, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fp8_prepare_forward(_addr(B, "B"), T, h, f, t, w, wn, _stream(stream)))
+
+
+def mlp_tp_fp8_prepare_backward(dY, X, A, B, T, h, f, t, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fp8_prepare_backward(_addr(dY, "dY", T == 0), _addr(X, "X", T == 0), _addr(A, "A"),
+                                             _addr(B, "B"), T, h, f, t, w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_forward_fp8(X, A, a, T, h, f, t, Z, H, H_lo, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_forward_fp8(_addr(X, "X", T == 0), _addr(A, "A"), _addr(a, "a"), T, h, f, t,
+                                        _addr(Z, "Z", T == 0), _addr(H, "H", T == 0, "f16"),
+                                        _addr(H_lo, "H_lo", T == 0, "e4m3"), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_forward_fp8(H, b, T, h, f, t, Y, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_forward_fp8(_addr(H, "H", T == 0, "f16"), _addr(b, "b", True), T, h, f, t,
+                                        _addr(Y, "Y", T == 0), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_backward_data_fp8(dY, B, Z, T, h, f, t, dH, dH_lo, da, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_backward_data_fp8(_addr(dY, "dY", T == 0), _addr(B, "B"), _addr(Z, "Z", T == 0),
+                                              T, h, f, t, _addr(dH, "dH", T == 0, "f16"),
+                                              _addr(dH_lo, "dH_lo", T == 0, "e4m3"), _addr(da, "da", True),
+                                              w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_backward_weight_fp8(H, H_lo, dY, T, h, f, t, dB, db, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_backward_weight_fp8(_addr(H, "H", T == 0, "f16"), _addr(H_lo, "H_lo", T == 0, "e4m3"),
+                                                _addr(dY, "dY", T == 0), T, h, f, t, _addr(dB, "dB"),
+                                                _addr(db, "db", True), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_data_fp8(dH, T, h, f, t, dX, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_data_fp8(_addr(dH, "dH", T == 0, "f16"), T, h, f, t, _addr(dX, "dX", T == 0),
+                                              w, wn, _stream(stream)))
+
+
+def mlp_tp_fc1_backward_weight_fp8(dH, dH_lo, T, h, f, t, dA, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_weight_fp8(_addr(dH, "dH", T == 0, "f16"),
+                                                _addr(dH_lo, "dH_lo", T == 0, "e4m3"), T, h, f, t,
+                                                _addr(dA, "dA"), w, wn, _stream(stream)))
 
 
 # ------------------------------------------------------------------ across GPUs

@@ -10,10 +10,18 @@ import torch
 from . import binding
 
 
-def alloc_outputs(T: int, h: int, f: int, device="cuda", with_bias_grads: bool = True) -> Dict[str, torch.Tensor]:
+def alloc_outputs(T: int, h: int, f: int, device="cuda", with_bias_grads: bool = True,
+                  mode: int = binding.ACCURATE) -> Dict[str, torch.Tensor]:
+    """Outputs and saved activations; in binding.FP8 mode H is fp16 and H_lo
+    holds the e4m3 residuals."""
     e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device=device)  # noqa: E731
-    out = {"Y": e(T, h), "Z": torch.empty(T, f, dtype=torch.float32, device=device), "H": e(T, f),
-           "H_lo": e(T, f), "dX": e(T, h), "dA": e(h, f), "dB": e(f, h)}
+    if mode == binding.FP8:
+        H = torch.empty(T, f, dtype=torch.float16, device=device)
+        H_lo = torch.empty(T, f, dtype=torch.float8_e4m3fn, device=device)
+    else:
+        H, H_lo = e(T, f), e(T, f)
+    out = {"Y": e(T, h), "Z": torch.empty(T, f, dtype=torch.float32, device=device), "H": H,
+           "H_lo": H_lo, "dX": e(T, h), "dA": e(h, f), "dB": e(f, h)}
     if with_bias_grads:
         out["da"] = e(f)
         out["db"] = e(h)
@@ -46,9 +54,9 @@ def forward_backward(inp: Dict[str, torch.Tensor], t: int, out: Optional[Dict[st
     f = inp["A"].shape[1]
     dev = inp["X"].device
     if out is None:
-        out = alloc_outputs(T, h, f, dev)
+        out = alloc_outputs(T, h, f, dev, mode=mode)
     if ws is None:
-        ws = binding.make_workspace(T, h, f, t, dev)
+        ws = binding.make_workspace_mode(T, h, f, t, mode, device=dev)
     forward(inp, t, out, ws, mode)
     backward(inp, t, out, ws, mode)
     if check:

@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "mlp_tp.cu")
 OUT = os.path.join(HERE, "libmlptp.so")
-DEPS = [os.path.join(HERE, "csrc", n) for n in ("mlp_tp.cu", "gemm.cuh", "ptx.cuh", "colsum.cuh", "peer.cuh", "peer_reduce.cuh")] + [
+DEPS = [os.path.join(HERE, "csrc", n) for n in ("mlp_tp.cu", "gemm.cuh", "ptx.cuh", "colsum.cuh", "fp8.cuh", "peer.cuh", "peer_reduce.cuh")] + [
     os.path.join(os.path.dirname(HERE), "include", "mlp_tp.h")]
 
 NVCC_FLAGS = [

@@ -50,6 +50,13 @@
 // 64 (rows) x 64 (K); the MMA reads it through an MN-major descriptor, so no
 // transpose is ever materialised.
 //
+// 8-bit residual products (F8LO).  In the fp16 + e4m3 mode (fp8.cuh) a
+// weight gradient is one fp16 product plus an e4m3 residual product into the
+// same accumulator.  The K loop runs the fp16 part (64-token stages) and then
+// the e4m3 part in stages of 128 tokens, which take the same bytes: A and B
+// arrive as 128 (rows) x 128 (K) boxes, 128-byte rows, and each stage issues
+// four kind::f8f6f4 MMAs of K = 32 per MMA width.
+//
 // Cross-GPU shard reduction (EPI_PEER).  With the block sharded over several
 // GPUs, a rank's row-parallel GEMM sends each 128-row block of its fp32
 // partial straight to the GPU that owns those token rows (peer.cuh): plain
@@ -66,6 +73,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "fp8.cuh"
 #include "peer.cuh"
 #include "ptx.cuh"
 
@@ -75,6 +83,7 @@ constexpr int BM = 128;  // accumulator rows per CTA
 constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
 constexpr int MN_BOX_BYTES = 64 * BK * 2;   // one 64x64 bf16 box, 8 KB
+constexpr int F8_BOX_BYTES = 128 * 2 * BK;  // one 128x128 e4m3 box, 16 KB
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int CTL_BYTES = 1024;
@@ -168,7 +177,8 @@ struct GemmParams {
   float* tail_scratch;    // [pieces][TILE_M][TILE_N] fp32
   long long scratch_elems;  // floats in tail_scratch (bounds-checking build)
   int parts;              // 1, or 2 when an operand is a bf16 (hi, lo) pair
-  int kblocks_per_shard;  // BK-wide K slices per segment and part
+  int kblocks_per_shard;  // BK-wide K slices per segment and part (F8LO: of the fp16 part)
+  int kb_per_unit;        // K slices (stages) per segment over all parts
   int m_blocks, n_blocks, num_tiles, group_m;
   __nv_bfloat16* out0;        // H_hi | Y | dH_hi | dX | dA | dB
   __nv_bfloat16* out1;        // H_lo (EPI_BIAS_GELU) | dH_lo (EPI_GELU_GRAD)
@@ -182,7 +192,30 @@ struct GemmParams {
   unsigned int debug_flags;
   PeerParams peer;            // EPI_PEER: where each row block's partial goes
   long long peer_recv_elems;  // floats in each receive buffer (bounds-checking build)
+  // fp16 + e4m3 mode (fp8.cuh)
+  uint32_t f16_ops;                // kind::f16 operands are fp16 (1) or bf16 (0)
+  const unsigned int* fp8_stats;   // the mode's statistics, from which the scales follow (NULL: none)
+  int out_scale;                   // OUT_SCALE_*: factor on the accumulator before the output rounding
+  int fp8_out;                     // EPI_BIAS_GELU / EPI_GELU_GRAD: out0 fp16, out1 e4m3 residual
 };
+
+enum OutScale : int { OUT_SCALE_NONE = 0, OUT_SCALE_INV_SY = 1, OUT_SCALE_INV_SX_SH = 2, OUT_SCALE_INV_SH = 3 };
+
+// The output factor that undoes the operands' power-of-two scales.
+__device__ __forceinline__ float out_factor(const GemmParams& p) {
+  if (p.fp8_stats == nullptr || p.out_scale == OUT_SCALE_NONE) return 1.0f;
+  const Fp8Scales sc = fp8_scales(p.fp8_stats);
+  if (p.out_scale == OUT_SCALE_INV_SY) return 1.0f / sc.sY;
+  if (p.out_scale == OUT_SCALE_INV_SX_SH) return 1.0f / (sc.sX * sc.sH);
+  return 1.0f / sc.sH;
+}
+
+__device__ __forceinline__ void record_range(const GemmParams& p, bool bad, unsigned int site) {
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) {
+    atomicCAS(p.status, 0u, STATUS_RANGE);
+    atomicCAS(p.status + 1, 0u, site);
+  }
+}
 
 // Tensor maps of the operands, one per K part (part 1 repeats part 0 for an
 // operand that is not split), and of the outputs (32x32 store boxes):
@@ -398,11 +431,13 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- kernel
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL, bool F8LO>
 __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
     mlp_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   static_assert(!DUAL || PAIR, "both halves of A in one stage: pair mode");
+  static_assert(!F8LO || (A_MN && B_MN && !DUAL && EPI == EPI_STORE),
+                "8-bit residual products: weight gradients over MN-major operands");
   static_assert(EPI != EPI_SHARD_SUM || TN == 256, "the shard sum is held in registers for 256 columns");
   static_assert(EPI != EPI_PEER || (TN == 256 && EW == PEER_ARRIVALS),
                 "a peer tile block is one MMA width and its arrival count is one per epilogue warp");
@@ -469,7 +504,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
   const uint64_t budget = p.budget_ns;
-  const int kb_per_unit = p.parts * p.kblocks_per_shard;
+  const int kb_per_unit = p.kb_per_unit;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -498,13 +533,44 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
               ok = false;
               break;
             }
-            const int part = i / p.kblocks_per_shard;
-            const int k0 = (s * p.kblocks_per_shard + (i - part * p.kblocks_per_shard)) * BK;
+            const bool f8 = F8LO && i >= p.kblocks_per_shard;  // an e4m3 stage of 2*BK tokens
+            const int part = F8LO ? (f8 ? 1 : 0) : i / p.kblocks_per_shard;
+            const int k0 = F8LO ? (f8 ? (i - p.kblocks_per_shard) * 2 * BK : i * BK)
+                                : (s * p.kblocks_per_shard + (i - part * p.kblocks_per_shard)) * BK;
             const CUtensorMap* ma = &maps.a[part];
             const CUtensorMap* mbp = &maps.b[part];
             const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
             const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
-            if constexpr (PAIR) {
+            if (f8) {
+              // same bytes as a 16-bit stage: A 128 x 128, B per MMA width SUB_ROWS x 128
+              uint32_t fb;
+              if constexpr (PAIR) {
+                fb = map_shared_to_cta(smem_u32(&ctl->full[stage]), 0u);
+                if (leader) mbar_arrive_expect_tx(&ctl->full[stage], Cfg::CTAS * Cfg::STAGE_BYTES);
+              } else {
+                fb = smem_u32(&ctl->full[stage]);
+                mbar_arrive_expect_tx(&ctl->full[stage], Cfg::STAGE_BYTES);
+              }
+              if (leader || !PAIR) {
+                issued_mask |= 1u << stage;
+                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+              }
+              if constexpr (PAIR) {
+                tma_load_2d_pair(a_dst, ma, fb, m0, k0);
+              } else {
+                tma_load_2d(a_dst, ma, fb, m0, k0);
+              }
+#pragma unroll
+              for (int w = 0; w < Cfg::WIDTHS; ++w)
+#pragma unroll
+                for (int j = 0; j < Cfg::SUB_ROWS / 128; ++j) {
+                  if constexpr (PAIR) {
+                    tma_load_2d_pair(b_dst + w * Cfg::SUB_BYTES + j * F8_BOX_BYTES, mbp, fb, n0 + w * BN + 128 * j, k0);
+                  } else {
+                    tma_load_2d(b_dst + w * Cfg::SUB_BYTES + j * F8_BOX_BYTES, mbp, fb, n0 + w * BN + 128 * j, k0);
+                  }
+                }
+            } else if constexpr (PAIR) {
               const uint32_t fb = map_shared_to_cta(smem_u32(&ctl->full[stage]), 0u);
               if (leader) {
                 mbar_arrive_expect_tx(&ctl->full[stage], Cfg::CTAS * Cfg::STAGE_BYTES);
@@ -575,7 +641,8 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(Cfg::TILE_M, BN, A_MN, B_MN);
+      const uint32_t IDESC = idesc_f32(Cfg::TILE_M, BN, A_MN, B_MN, p.f16_ops ? FMT_F16 : FMT_BF16);
+      constexpr uint32_t IDESC8 = idesc_f32(Cfg::TILE_M, BN, A_MN, B_MN, FMT_E4M3);
       constexpr uint16_t PAIR_MASK = 0x3;
       int stage = 0;
       uint32_t phase = 0, unit = 0;
@@ -600,6 +667,25 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             tc_fence_after_sync();
             const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
             const uint32_t b_base = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+            if (F8LO && i >= p.kblocks_per_shard) {
+              // e4m3 stage: 128 K rows of 128 bytes; each MMA takes K = 32
+              // rows (4 groups of 8, 4096 bytes); 128-row MN blocks are one
+              // 16 KB box apart
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = smem_desc_sw128(a_base + k * 4096, F8_BOX_BYTES, 1024);
+#pragma unroll
+                for (int w = 0; w < Cfg::WIDTHS; ++w) {
+                  const uint64_t bd = smem_desc_sw128(b_base + w * Cfg::SUB_BYTES + k * 4096, F8_BOX_BYTES, 1024);
+                  const uint32_t accumulate = (i != it.i_begin || k != 0) ? 1u : 0u;
+                  if constexpr (PAIR) {
+                    mma_f8_pair(d_tmem + w * BN, ad, bd, IDESC8, accumulate);
+                  } else {
+                    mma_f8_ss(d_tmem + w * BN, ad, bd, IDESC8, accumulate);
+                  }
+                }
+              }
+            } else {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
               // K-major: the 16-wide K slice is 32 bytes further along each
@@ -626,6 +712,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
                   mma_bf16_ss(d_tmem + w * BN, ad, bd, IDESC, accumulate);
                 }
               }
+            }
             }
             if constexpr (PAIR) {
               mma_commit_pair_multicast(&ctl->empty[stage], PAIR_MASK);
@@ -665,6 +752,10 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
     const uint32_t st_f32 = stage_base;
     const uint32_t st_out0 = stage_base + (EPI == EPI_BIAS_GELU ? EPI_F32_TILE : 0);
     const uint32_t st_out1 = st_out0 + EPI_BF16_TILE;
+    // fp16 + e4m3 mode: the factor that undoes the operands' scales, and the
+    // scale of dH (EPI_GELU_GRAD)
+    const float out_mul = out_factor(p);
+    const float s_dh = p.fp8_stats != nullptr ? fp8_scales(p.fp8_stats).sH : 1.0f;
     uint32_t tempty_addr[2] = {0u, 0u};
     if constexpr (PAIR) {
 #pragma unroll
@@ -745,11 +836,30 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             uint32_t hp[16], lp[16];
 #pragma unroll
             for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(r[j]) + bias[j];
+            if (p.fp8_out) {
+              // H as fp16 plus its e4m3 residual (H − fp16(H))·2^7
+              bool big = false;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) split_bf16x2(gelu_f(z[2 * j]), gelu_f(z[2 * j + 1]), hp[j], lp[j]);
-            stage_f32x32(st_f32, lane, z);
-            stage_bf16x32(st_out0, lane, hp);
-            stage_bf16x32(st_out1, lane, lp);
+              for (int j = 0; j < 8; ++j) lp[j] = 0u;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float g0 = gelu_f(z[2 * j]), g1 = gelu_f(z[2 * j + 1]);
+                big |= fabsf(g0) >= FP8_H_LIMIT || fabsf(g1) >= FP8_H_LIMIT;
+                uint32_t lo8;
+                split_f16_e4m3(g0, g1, hp[j], lo8);
+                lp[j >> 1] |= lo8 << (16 * (j & 1));
+              }
+              record_range(p, big, 0xB01u);
+              stage_f32x32(st_f32, lane, z);
+              stage_bf16x32(st_out0, lane, hp);  // fp16: same 64-byte rows and swizzle
+              stage_e4m3x32(st_out1, lane, reinterpret_cast<const uint32_t(&)[8]>(lp));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) split_bf16x2(gelu_f(z[2 * j]), gelu_f(z[2 * j + 1]), hp[j], lp[j]);
+              stage_f32x32(st_f32, lane, z);
+              stage_bf16x32(st_out0, lane, hp);
+              stage_bf16x32(st_out1, lane, lp);
+            }
             fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0) {
@@ -766,10 +876,28 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) dh[j] = row_ok ? __uint_as_float(r[j]) * gelu_grad_f(z[j]) : 0.0f;
             uint32_t hp[16], lp[16];
+            if (p.fp8_out) {
+              // dH·sH as fp16 plus its e4m3 residual
+              bool big = false;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) split_bf16x2(dh[2 * j], dh[2 * j + 1], hp[j], lp[j]);
-            stage_bf16x32(st_out0, lane, hp);
-            stage_bf16x32(st_out1, lane, lp);
+              for (int j = 0; j < 8; ++j) lp[j] = 0u;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float d0 = dh[2 * j] * s_dh, d1 = dh[2 * j + 1] * s_dh;
+                big |= fabsf(d0) >= FP8_H_LIMIT || fabsf(d1) >= FP8_H_LIMIT;
+                uint32_t lo8;
+                split_f16_e4m3(d0, d1, hp[j], lo8);
+                lp[j >> 1] |= lo8 << (16 * (j & 1));
+              }
+              record_range(p, big, 0xB02u);
+              stage_bf16x32(st_out0, lane, hp);
+              stage_e4m3x32(st_out1, lane, reinterpret_cast<const uint32_t(&)[8]>(lp));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) split_bf16x2(dh[2 * j], dh[2 * j + 1], hp[j], lp[j]);
+              stage_bf16x32(st_out0, lane, hp);
+              stage_bf16x32(st_out1, lane, lp);
+            }
             fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0) {
@@ -821,7 +949,8 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             }
             uint32_t op[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) op[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            for (int j = 0; j < 16; ++j)
+              op[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * out_mul, __uint_as_float(r[2 * j + 1]) * out_mul);
             stage_bf16x32(st_out0, lane, op);
             fence_proxy_async_shared();
             __syncwarp();
@@ -860,7 +989,8 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
               uint32_t yp[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j)
-                yp[j] = pack_bf16x2(sum[c * 32 + 2 * j] + bias[2 * j], sum[c * 32 + 2 * j + 1] + bias[2 * j + 1]);
+                yp[j] = pack_bf16x2(fmaf(sum[c * 32 + 2 * j], out_mul, bias[2 * j]),
+                                    fmaf(sum[c * 32 + 2 * j + 1], out_mul, bias[2 * j + 1]));
               stage_bf16x32(st_out0, lane, yp);
               fence_proxy_async_shared();
               __syncwarp();
@@ -944,6 +1074,9 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const GemmParams p, i
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = part == 0 ? v[e] : acc[e] + v[e];
   }
+  const float mul = out_factor(p);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] *= mul;
   float bias[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) bias[e] = 0.0f;

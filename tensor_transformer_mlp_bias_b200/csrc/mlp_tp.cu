@@ -14,6 +14,7 @@
 
 #include "../../include/mlp_tp.h"
 #include "colsum.cuh"
+#include "fp8.cuh"
 #include "gemm.cuh"
 #include "peer_reduce.cuh"
 
@@ -178,6 +179,29 @@ size_t recompute_h_offset(const Shape& s) {
 size_t recompute_hlo_offset(const Shape& s) { return recompute_h_offset(s) + pair_bytes(s); }
 size_t recompute_workspace_bytes(const Shape& s) { return recompute_hlo_offset(s) + pair_bytes(s); }
 
+// The fp16 + e4m3 mode keeps its operand copies after the rest of the
+// workspace: [ ... | W16 (fp16 copy of B in the forward, of A in the
+// backward) | X16 | X8 | dY16 | dY8 ], and its statistics in the header.
+constexpr size_t FP8_STATS_OFFSET = 64;
+struct Fp8Layout {
+  size_t w16, x16, x8, dy16, dy8, bytes;
+};
+Fp8Layout fp8_layout(const Shape& s) {
+  Fp8Layout l;
+  const size_t th = static_cast<size_t>(s.T * s.h), hf = static_cast<size_t>(s.h * s.f);
+  l.w16 = 0;
+  l.x16 = l.w16 + align_up(hf * 2, 256);
+  l.x8 = l.x16 + align_up(th * 2, 256);
+  l.dy16 = l.x8 + align_up(th, 256);
+  l.dy8 = l.dy16 + align_up(th * 2, 256);
+  l.bytes = l.dy8 + align_up(th, 256);
+  return l;
+}
+size_t mode_workspace_bytes(const Shape& s, int32_t mode, bool recompute) {
+  const size_t base = recompute ? recompute_workspace_bytes(s) : workspace_bytes(s);
+  return base + (mode == MLP_TP_FP8 ? fp8_layout(s).bytes : 0);
+}
+
 struct Ptr {
   const void* p;
   const char* name;
@@ -197,10 +221,10 @@ mlp_status_t check_ptrs(std::initializer_list<Ptr> ptrs) {
   return MLP_OK;
 }
 
-mlp_status_t check_ws(const Shape& s, void* ws, size_t ws_bytes, bool recompute = false) {
+mlp_status_t check_ws(const Shape& s, void* ws, size_t ws_bytes, bool recompute = false, int32_t mode = 0) {
   if (ws == nullptr) return fail(MLP_ERR_INVALID_ARG, "workspace pointer is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MLP_ERR_MISALIGNED, "workspace is not 256-byte aligned");
-  const size_t need = recompute ? recompute_workspace_bytes(s) : workspace_bytes(s);
+  const size_t need = mode_workspace_bytes(s, mode, recompute);
   if (ws_bytes < need)
     return fail(MLP_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
   return MLP_OK;
@@ -260,11 +284,14 @@ EncodeTiledFn encode_fn() {
 // swizzle, so an entry whose key matches all of those is the map the driver
 // would encode again; a launch-bound step (small batches) spends much of its
 // host time encoding about seven maps per GEMM otherwise.
+// Element formats of operands and outputs.
+enum OpFmt : int { OP_BF16 = 0, OP_F16 = 1, OP_E4M3 = 2, OP_F32 = 3 };
+
 struct MapKey {
   const void* ptr;
   int64_t rows, cols;
   uint32_t box0, box1;
-  int kind;  // 0: bf16 operand (128-byte swizzle), 1: bf16 output (64-byte), 2: fp32 output (128-byte)
+  int kind;  // operand: OpFmt (128-byte swizzle); output: 16 + OpFmt
   bool operator==(const MapKey& o) const {
     return ptr == o.ptr && rows == o.rows && cols == o.cols && box0 == o.box0 && box1 == o.box1 && kind == o.kind;
   }
@@ -292,19 +319,24 @@ struct MapCache {
 };
 thread_local MapCache g_map_cache;
 
-// 2-D bf16 row-major matrix [rows, cols] (cols contiguous), box of
-// 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+// 2-D row-major operand [rows, cols] (cols contiguous), box of 128 bytes of
+// columns (64 16-bit or 128 8-bit values) x box_rows rows, 128-byte swizzle,
+// zero fill out of bounds.
 mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, uint32_t box_rows,
-                      const char* name) {
-  const MapKey key{ptr, rows, cols, 64u, box_rows, 0};
+                      const char* name, int fmt = OP_BF16) {
+  const cuuint64_t esz = fmt == OP_E4M3 ? 1 : 2;
+  const uint32_t box_cols = static_cast<uint32_t>(128 / esz);
+  const MapKey key{ptr, rows, cols, box_cols, box_rows, fmt};
   if (g_map_cache.find(key, map)) return MLP_OK;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64u, box_rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esz};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  const CUtensorMapDataType dt = fmt == OP_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : (fmt == OP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for %s (CUresult %d)", name, (int)r);
@@ -313,22 +345,27 @@ mlp_status_t make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t c
 }
 
 // Output of a GEMM epilogue: row-major [rows, cols], stored in 32x32 boxes
-// from the epilogue's swizzled staging tiles (bf16: 64-byte swizzle, fp32:
-// 128-byte swizzle, matching the staging layout in gemm.cuh).
-mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, bool f32, const char* name) {
-  const MapKey key{ptr, rows, cols, 32u, 32u, f32 ? 2 : 1};
+// from the epilogue's swizzled staging tiles (bf16, fp16: 64-byte swizzle;
+// fp32: 128-byte; e4m3: 32-byte; matching the staging layouts in gemm.cuh
+// and fp8.cuh).
+mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int fmt, const char* name) {
+  const MapKey key{ptr, rows, cols, 32u, 32u, 16 + fmt};
   if (g_map_cache.find(key, map)) return MLP_OK;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t esz = f32 ? 4 : 2;
+  const cuuint64_t esz = fmt == OP_F32 ? 4 : (fmt == OP_E4M3 ? 1 : 2);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esz};
   cuuint32_t box[2] = {32u, 32u};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = fmt == OP_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : fmt == OP_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : fmt == OP_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = fmt == OP_F32 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : (fmt == OP_E4M3 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+  CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MLP_ERR_CUDA, "cuTensorMapEncodeTiled failed for output of %s (CUresult %d)", name, (int)r);
   g_map_cache.put(key, *map);
@@ -336,17 +373,20 @@ mlp_status_t make_out_map(CUtensorMap* map, const void* ptr, int64_t rows, int64
 }
 
 // Operand of the GEMM: `rows` is its M (or N) extent, `k` its K extent.
-// K-major: stored [rows, k];  MN-major: stored [k, rows].
+// K-major: stored [rows, k];  MN-major: stored [k, rows].  e4m3 operands are
+// MN-major only, in 128 x 128 boxes (the 8-bit stages of F8LO).
 mlp_status_t make_operand_map(CUtensorMap* map, const void* ptr, bool mn_major, int64_t rows, int64_t k,
-                              uint32_t tile_rows, const char* name) {
-  if (mn_major) return make_map(map, ptr, k, rows, 64u, name);
-  return make_map(map, ptr, rows, k, tile_rows, name);
+                              uint32_t tile_rows, const char* name, int fmt) {
+  if (fmt == OP_E4M3) return make_map(map, ptr, k, rows, 128u, name, fmt);
+  if (mn_major) return make_map(map, ptr, k, rows, 64u, name, fmt);
+  return make_map(map, ptr, rows, k, tile_rows, name, fmt);
 }
 
 // ---------------------------------------------------------------- launches
 struct Operand {
   const void* p[2];  // part 0 and part 1 (part 1 = part 0 when not split)
   bool mn_major;
+  int fmt[2] = {OP_BF16, OP_BF16};
 };
 
 struct GemmDesc {
@@ -373,13 +413,13 @@ int pick_group_m(int64_t M, int64_t N, int64_t K, int m_blocks) {
 
 // One opt-in per kernel instantiation and device (the static state is per
 // template instance).
-template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL>
+template <bool A_MN, bool B_MN, int EPI, bool PAIR, int TN, int EW, bool DUAL, bool F8LO>
 mlp_status_t ensure_kernel_setup(int dev, int sms, int* max_clusters) {
   using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   static std::mutex mu;
   static uint64_t done_mask = 0;
   static int clusters[64] = {};
-  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>;
+  auto kernel = mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL, F8LO>;
   std::lock_guard<std::mutex> lk(mu);
   if (!(done_mask & (1ull << dev))) {
     cudaError_t e =
@@ -435,23 +475,26 @@ cudaError_t launch_helper(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaS
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
-template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8, bool DUAL = false>
+template <bool A_MN, bool B_MN, int EPI, int TN = 256, bool PAIR = kPair, int EW = 8, bool DUAL = false,
+          bool F8LO = false>
 mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const char* name) {
   using Cfg = TileCfg<PAIR, TN, EPI, EW, DUAL>;
   if (g.M == 0 || g.N == 0) return MLP_OK;
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   {
-    // EPI_PEER stores with plain instructions and has no output tensor map
-    mlp_status_t st = p.out0 != nullptr ? make_out_map(&maps.out[0], p.out0, g.M, g.N, false, name) : MLP_OK;
-    if (st == MLP_OK && p.out1 != nullptr) st = make_out_map(&maps.out[1], p.out1, g.M, g.N, false, name);
-    if (st == MLP_OK && p.out_f32 != nullptr) st = make_out_map(&maps.out[2], p.out_f32, g.M, g.N, true, name);
+    // EPI_PEER stores with plain instructions and has no output tensor map;
+    // with fp8_out the pair is (fp16, e4m3 residual)
+    const int f0 = p.fp8_out ? OP_F16 : OP_BF16, f1 = p.fp8_out ? OP_E4M3 : OP_BF16;
+    mlp_status_t st = p.out0 != nullptr ? make_out_map(&maps.out[0], p.out0, g.M, g.N, f0, name) : MLP_OK;
+    if (st == MLP_OK && p.out1 != nullptr) st = make_out_map(&maps.out[1], p.out1, g.M, g.N, f1, name);
+    if (st == MLP_OK && p.out_f32 != nullptr) st = make_out_map(&maps.out[2], p.out_f32, g.M, g.N, OP_F32, name);
     if (st != MLP_OK) return st;
   }
   for (int i = 0; i < 2; ++i) {
-    mlp_status_t st = make_operand_map(&maps.a[i], g.a.p[i], A_MN, g.M, g.K, BM, name);
+    mlp_status_t st = make_operand_map(&maps.a[i], g.a.p[i], A_MN, g.M, g.K, BM, name, g.a.fmt[i]);
     if (st != MLP_OK) return st;
-    st = make_operand_map(&maps.b[i], g.b.p[i], B_MN, g.N, g.K, Cfg::SUB_ROWS, name);
+    st = make_operand_map(&maps.b[i], g.b.p[i], B_MN, g.N, g.K, Cfg::SUB_ROWS, name, g.b.fmt[i]);
     if (st != MLP_OK) return st;
   }
   p.M = static_cast<int>(g.M);
@@ -459,6 +502,9 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.shards = g.shards;
   p.parts = DUAL ? 1 : g.parts;  // DUAL: both halves of A in each stage, one pass over K
   p.kblocks_per_shard = static_cast<int>((g.K / g.shards + BK - 1) / BK);
+  // F8LO: the fp16 part in BK-token stages, then the e4m3 part in 2*BK-token stages
+  p.kb_per_unit = F8LO ? p.kblocks_per_shard + static_cast<int>((g.K + 2 * BK - 1) / (2 * BK))
+                       : p.parts * p.kblocks_per_shard;
   p.m_blocks = static_cast<int>((g.M + Cfg::TILE_M - 1) / Cfg::TILE_M);
   p.n_blocks = static_cast<int>((g.N + Cfg::TILE_N - 1) / Cfg::TILE_N);
   p.num_tiles = p.m_blocks * p.n_blocks;
@@ -466,7 +512,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.debug_flags = g_debug_flags.load();
 
   int max_clusters = 0;
-  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>(L.dev, L.sms, &max_clusters);
+  mlp_status_t st = ensure_kernel_setup<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL, F8LO>(L.dev, L.sms, &max_clusters);
   if (st != MLP_OK) return st;
   p.group_m = pick_group_m(g.M, g.N, g.K, p.m_blocks);
   // Work list.  Split pieces trade idle CTA pairs for extra traffic: a piece
@@ -487,7 +533,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   p.kb_split = 1;
   const size_t piece_bytes = static_cast<size_t>(Cfg::TILE_M) * Cfg::TILE_N * sizeof(float);
   const size_t capacity = g.tail_scratch != nullptr ? g.tail_bytes / piece_bytes : 0;
-  const int kb_per_unit = p.parts * p.kblocks_per_shard;  // slices per shard
+  const int kb_per_unit = p.kb_per_unit;  // slices per shard
   auto rounds = [&](long long items) { return static_cast<double>((items + max_clusters - 1) / max_clusters); };
   // weight gradients: at least enough pieces to keep each accumulator within
   // kWgradMaxAdds additions (long token axes)
@@ -552,7 +598,7 @@ mlp_status_t launch_gemm(const GemmDesc& g, GemmParams p, const Launch& L, const
   cfg.stream = L.stream;
   cfg.attrs = attr;
   cfg.numAttrs = PAIR ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL>, maps, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mlp_gemm_kernel<A_MN, B_MN, EPI, PAIR, TN, EW, DUAL, F8LO>, maps, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, name);
   g_launches.fetch_add(1);
@@ -634,6 +680,8 @@ mlp_status_t read_status_word(unsigned int* status, cudaStream_t cs) {
     return fail(MLP_ERR_TIMEOUT, "a kernel wait ran out of its budget (site 0x%x)", word[1]);
   if (word[0] == STATUS_BOUNDS)
     return fail(MLP_ERR_BOUNDS, "an index fell outside its buffer (site 0x%x; bounds-checking build)", word[1]);
+  if (word[0] == STATUS_RANGE)
+    return fail(MLP_ERR_RANGE, "a value outside the range of the fp16 + e4m3 mode (site 0x%x)", word[1]);
   return fail(MLP_ERR_CUDA, "device status word holds unknown code %u", word[0]);
 }
 
@@ -737,6 +785,212 @@ mlp_status_t fc1_backward_weight(const Shape& s, const void* X, const void* dH, 
   return launch_gemm<true, true, EPI_STORE, kWideTN>(g, p, L, "column-parallel weight gradient (dA)");
 }
 
+// ---------------------------------------------------------------- fp16 + e4m3 mode
+// (fp8.cuh).  The forward casts B to fp16; the backward reduces the
+// statistics the scales follow from and casts X, dY (fp16 and e4m3, scaled)
+// and A (fp16); the GEMMs then run on those copies.
+struct Fp8Bufs {
+  void* w16;
+  void* x16;
+  void* x8;
+  void* dy16;
+  void* dy8;
+  unsigned int* stats;
+};
+
+Fp8Bufs fp8_bufs(void* ws, const Shape& s, bool recompute) {
+  char* w = static_cast<char*>(ws);
+  char* r = w + (recompute ? recompute_workspace_bytes(s) : workspace_bytes(s));
+  const Fp8Layout l = fp8_layout(s);
+  return Fp8Bufs{r + l.w16, r + l.x16, r + l.x8, r + l.dy16, r + l.dy8,
+                 reinterpret_cast<unsigned int*>(w + FP8_STATS_OFFSET)};
+}
+
+mlp_status_t launch_cast(const CastJobs& jobs, const unsigned int* stats, void* ws, const Launch& L) {
+  long long n = 0;
+  for (int j = 0; j < jobs.count; ++j) n += jobs.job[j].n;
+  if (n == 0) return MLP_OK;
+  cudaError_t e = launch_helper(fp8_cast_kernel, dim3(static_cast<unsigned>(L.sms * 4)), dim3(256), L.stream, jobs,
+                                stats, static_cast<unsigned int*>(ws));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_cast");
+  g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+// B -> fp16 copy (W16), for the row-parallel forward.
+mlp_status_t fp8_prepare_forward(const Shape& s, const void* B, const Fp8Bufs& q, void* ws, const Launch& L) {
+  CastJobs jobs;
+  memset(&jobs, 0, sizeof(jobs));
+  jobs.job[0] = CastJob{static_cast<const __nv_bfloat16*>(B), static_cast<__half*>(q.w16), nullptr, s.f * s.h,
+                        CAST_UNSCALED};
+  jobs.count = 1;
+  return launch_cast(jobs, nullptr, ws, L);
+}
+
+// Statistics of X, dY and B, then X -> (X16, X8), dY -> (dY16, dY8) and
+// A -> W16.
+mlp_status_t fp8_prepare_backward(const Shape& s, const void* dY, const void* X, const void* A, const void* B,
+                                  const Fp8Bufs& q, void* ws, const Launch& L) {
+  mlp_status_t st = zero_fill(q.stats, STAT_WORDS * sizeof(unsigned int), L.stream, "cudaMemsetAsync(fp8 statistics)");
+  if (st != MLP_OK) return st;
+  const long long rows = 2LL * s.T + s.f;
+  const long long want = (rows + STATS_THREADS / 32 - 1) / (STATS_THREADS / 32);
+  const long long blocks = want < 4LL * L.sms ? want : 4LL * L.sms;
+  cudaError_t e = launch_helper(fp8_stats_kernel, dim3(static_cast<unsigned>(blocks)), dim3(STATS_THREADS), L.stream,
+                                static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(dY),
+                                static_cast<const __nv_bfloat16*>(B), static_cast<int>(s.T), static_cast<int>(s.h),
+                                static_cast<int>(s.f), q.stats);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_stats");
+  g_launches.fetch_add(1);
+  CastJobs jobs;
+  memset(&jobs, 0, sizeof(jobs));
+  jobs.job[0] = CastJob{static_cast<const __nv_bfloat16*>(X), static_cast<__half*>(q.x16),
+                        static_cast<uint8_t*>(q.x8), s.T * s.h, CAST_SX};
+  jobs.job[1] = CastJob{static_cast<const __nv_bfloat16*>(dY), static_cast<__half*>(q.dy16),
+                        static_cast<uint8_t*>(q.dy8), s.T * s.h, CAST_SY};
+  jobs.job[2] = CastJob{static_cast<const __nv_bfloat16*>(A), static_cast<__half*>(q.w16), nullptr, s.h * s.f,
+                        CAST_UNSCALED};
+  jobs.count = 3;
+  return launch_cast(jobs, q.stats, ws, L);
+}
+
+Operand op16(const void* p, bool mn) { return Operand{{p, p}, mn, {OP_F16, OP_F16}}; }
+Operand op16_8(const void* p16, const void* p8, bool mn) { return Operand{{p16, p8}, mn, {OP_F16, OP_E4M3}}; }
+
+// Z = X·A + a (fp32), H16 = fp16(g(Z)), H8 = e4m3((g(Z) − H16)·2^7).
+mlp_status_t fc1_forward_fp8(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H16,
+                             void* H8, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.out_f32 = static_cast<float*>(Z);
+  p.out0 = static_cast<__nv_bfloat16*>(H16);
+  p.out1 = static_cast<__nv_bfloat16*>(H8);
+  p.bias = static_cast<const __nv_bfloat16*>(a);
+  p.fp8_out = 1;
+  GemmDesc g{one(X, false), one(A, true), s.T, s.f, s.h, 1, 1};
+  if (kFc1TN == 512) {
+    const int pairs = L.sms / TileShape::CTAS;
+    const int64_t mt = (s.T + TileShape::TILE_M - 1) / TileShape::TILE_M;
+    auto wave_eff = [&](int64_t tn) {
+      const int64_t tiles = mt * ((s.f + tn - 1) / tn);
+      const int64_t waves = (tiles + pairs - 1) / pairs;
+      return static_cast<double>(tiles) / static_cast<double>(waves * pairs);
+    };
+    const int64_t tiles256 = mt * ((s.f + 255) / 256);
+    if (tiles256 > pairs && wave_eff(512) + 0.05 >= wave_eff(256))
+      return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H16, H8)");
+  }
+  return launch_gemm<false, true, EPI_BIAS_GELU, 256>(g, p, L, "column-parallel forward (Z, H16, H8)");
+}
+
+// Y = Σ_i H16_i·B16_i + b.
+mlp_status_t fc2_forward_fp8(const Shape& s, const void* H16, const void* B16, const void* b, void* Y, void* ws,
+                             const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(Y);
+  p.bias = static_cast<const __nv_bfloat16*>(b);
+  p.f16_ops = 1;
+  GemmDesc g{op16(H16, false), op16(B16, true), s.T, s.h, s.f, s.t, 1, tail_scratch(ws, s), split_scratch_bytes(s)};
+  return launch_gemm<false, true, EPI_SHARD_SUM>(g, p, L, "row-parallel forward + shard reduce (Y, fp16)");
+}
+
+// dH = (dY·Bᵀ) ⊙ g'(Z) in fp32; dH16 = fp16(dH·sH), dH8 = e4m3((dH·sH − dH16)·2^7); da from the fp32 dH.
+mlp_status_t fc2_backward_data_fp8(const Shape& s, const void* dY, const void* B, const void* Z, void* dH16,
+                                   void* dH8, void* da, const unsigned int* stats, void* ws, const Launch& L) {
+  if (s.T == 0) return da != nullptr ? zero_fill(da, static_cast<size_t>(s.f) * 2, L.stream, "cudaMemsetAsync(da)")
+                                     : MLP_OK;
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dH16);
+  p.out1 = static_cast<__nv_bfloat16*>(dH8);
+  p.aux = static_cast<const float*>(Z);
+  p.colsum = da != nullptr ? partials(ws, s) : nullptr;
+  p.colsum_elems = static_cast<long long>(partial_bytes(s) / sizeof(float));
+  p.fp8_out = 1;
+  p.fp8_stats = stats;
+  GemmDesc g{one(dY, false), one(B, false), s.T, s.f, s.h, 1, 1};
+  mlp_status_t st =
+      s.h <= kFc2BdManyWarpsMaxK
+          ? launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 16>(g, p, L, "row-parallel backward data (dH16, dH8, da)")
+          : launch_gemm<false, false, EPI_GELU_GRAD, kFc2BdTN, kPair, 8>(g, p, L, "row-parallel backward data (dH16, dH8, da)");
+  if (st != MLP_OK || da == nullptr) return st;
+  return launch_colsum_final(partials(ws, s), static_cast<int>(gemm_row_blocks(s.T) * 4), s.f, da, L.stream,
+                             partial_bytes(s) / sizeof(float), static_cast<unsigned int*>(ws));
+}
+
+// dB = (H16ᵀ·dY16 + H8ᵀ·dY8) / sY, db = Σ_rows dY.
+mlp_status_t fc2_backward_weight_fp8(const Shape& s, const void* H16, const void* H8, const void* dY16,
+                                     const void* dY8, const void* dY, void* dB, void* db, const unsigned int* stats,
+                                     void* ws, const Launch& L) {
+  mlp_status_t st;
+  if (s.T == 0) {
+    st = zero_fill(dB, static_cast<size_t>(s.f * s.h * 2), L.stream, "cudaMemsetAsync(dB)");
+  } else {
+    GemmParams p = base_params(ws);
+    p.out0 = static_cast<__nv_bfloat16*>(dB);
+    p.f16_ops = 1;
+    p.fp8_stats = stats;
+    p.out_scale = OUT_SCALE_INV_SY;
+    GemmDesc g{op16_8(H16, H8, true), op16_8(dY16, dY8, true), s.f, s.h, s.T, 1, 2, tail_scratch(ws, s),
+               split_scratch_bytes(s)};
+    st = launch_gemm<true, true, EPI_STORE, kWideTN, kPair, 8, false, true>(
+        g, p, L, "row-parallel weight gradient (dB, fp16 + e4m3)");
+  }
+  if (st != MLP_OK || db == nullptr) return st;
+  return launch_colsum(dY, s.T, s.h, db, partials(ws, s), L.stream, partial_bytes(s) / sizeof(float),
+                       static_cast<unsigned int*>(ws));
+}
+
+// dX = (Σ_i dH16_i·A16_iᵀ) / sH.
+mlp_status_t fc1_backward_data_fp8(const Shape& s, const void* dH16, const void* A16, void* dX,
+                                   const unsigned int* stats, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dX);
+  p.f16_ops = 1;
+  p.fp8_stats = stats;
+  p.out_scale = OUT_SCALE_INV_SH;
+  GemmDesc g{op16(dH16, false), op16(A16, false), s.T, s.h, s.f, s.t, 1, tail_scratch(ws, s), split_scratch_bytes(s)};
+  return launch_gemm<false, false, EPI_SHARD_SUM>(g, p, L, "column-parallel backward data + shard reduce (dX, fp16)");
+}
+
+// dA = (X16ᵀ·dH16 + X8ᵀ·dH8) / (sX·sH).
+mlp_status_t fc1_backward_weight_fp8(const Shape& s, const void* X16, const void* X8, const void* dH16,
+                                     const void* dH8, void* dA, const unsigned int* stats, void* ws, const Launch& L) {
+  if (s.T == 0) return zero_fill(dA, static_cast<size_t>(s.h * s.f * 2), L.stream, "cudaMemsetAsync(dA)");
+  GemmParams p = base_params(ws);
+  p.out0 = static_cast<__nv_bfloat16*>(dA);
+  p.f16_ops = 1;
+  p.fp8_stats = stats;
+  p.out_scale = OUT_SCALE_INV_SX_SH;
+  GemmDesc g{op16_8(X16, X8, true), op16_8(dH16, dH8, true), s.h, s.f, s.T, 1, 2, tail_scratch(ws, s),
+             split_scratch_bytes(s)};
+  return launch_gemm<true, true, EPI_STORE, kWideTN, kPair, 8, false, true>(
+      g, p, L, "column-parallel weight gradient (dA, fp16 + e4m3)");
+}
+
+// The whole fp16 + e4m3 backward, given the saved Z, H16, H8; dH16 and dH8
+// live in the dH pair's slots of the workspace.
+mlp_status_t backward_fp8(const Shape& s, const void* dY, const void* X, const void* A, const void* B, const void* Z,
+                          const void* H16, const void* H8, void* dX, void* dA, void* da, void* dB, void* db, void* ws,
+                          bool recompute, const Launch& L) {
+  const Fp8Bufs q = fp8_bufs(ws, s, recompute);
+  void* dH16 = static_cast<char*>(ws) + dh_offset();
+  void* dH8 = static_cast<char*>(ws) + dh_lo_offset(s);
+  mlp_status_t st;
+  if ((st = fp8_prepare_backward(s, dY, X, A, B, q, ws, L)) != MLP_OK) return st;
+  if ((st = fc2_backward_data_fp8(s, dY, B, Z, dH16, dH8, da, q.stats, ws, L)) != MLP_OK) return st;
+  if ((st = fc2_backward_weight_fp8(s, H16, H8, q.dy16, q.dy8, dY, dB, db, q.stats, ws, L)) != MLP_OK) return st;
+  if ((st = fc1_backward_data_fp8(s, dH16, q.w16, dX, q.stats, ws, L)) != MLP_OK) return st;
+  return fc1_backward_weight_fp8(s, q.x16, q.x8, dH16, dH8, dA, q.stats, ws, L);
+}
+
+mlp_status_t forward_fp8(const Shape& s, const void* X, const void* A, const void* a, const void* B, const void* b,
+                         void* Y, void* Z, void* H16, void* H8, void* ws, bool recompute, const Launch& L) {
+  const Fp8Bufs q = fp8_bufs(ws, s, recompute);
+  mlp_status_t st;
+  if ((st = fp8_prepare_forward(s, B, q, ws, L)) != MLP_OK) return st;
+  if ((st = fc1_forward_fp8(s, X, A, a, Z, H16, H8, ws, L)) != MLP_OK) return st;
+  return fc2_forward_fp8(s, H16, q.w16, b, Y, ws, L);
+}
+
 // ---------------------------------------------------------------- across GPUs
 // Buffers and tile blocks of the cross-GPU shard reduction (peer.cuh).
 struct PeerShape {
@@ -813,19 +1067,19 @@ mlp_status_t fc1_backward_data_peer(const Shape& s, const void* dH, const void* 
 
 // Common preamble: shape, pointers, workspace, device.
 mlp_status_t prologue(const Shape& s, std::initializer_list<Ptr> ptrs, void* ws, size_t ws_bytes, void* stream,
-                      Launch& L, bool recompute = false) {
+                      Launch& L, bool recompute = false, int32_t mode = 0) {
   mlp_status_t st = check_shape(s);
   if (st != MLP_OK) return st;
   st = check_ptrs(ptrs);
   if (st != MLP_OK) return st;
-  st = check_ws(s, ws, ws_bytes, recompute);
+  st = check_ws(s, ws, ws_bytes, recompute, mode);
   if (st != MLP_OK) return st;
   L.stream = static_cast<cudaStream_t>(stream);
   return current_device(L.dev, L.sms);
 }
 
 mlp_status_t check_mode(int32_t mode) {
-  if (mode < MLP_TP_ACCURATE || mode > MLP_TP_FAST) return fail(MLP_ERR_INVALID_ARG, "precision mode %d out of range", mode);
+  if (mode < MLP_TP_ACCURATE || mode > MLP_TP_FP8) return fail(MLP_ERR_INVALID_ARG, "precision mode %d out of range", mode);
   return MLP_OK;
 }
 
@@ -882,8 +1136,9 @@ mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a, const v
   if (st != MLP_OK) return st;
   st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
                     {Y, "Y", false, s.T == 0}, {Z, "Z", false, s.T == 0}, {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}},
-                ws, ws_bytes, stream, L);
+                ws, ws_bytes, stream, L, false, mode);
   if (st != MLP_OK) return st;
+  if (mode == MLP_TP_FP8) return forward_fp8(s, X, A, a, B, b, Y, Z, H, H_lo, ws, false, L);
   st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L);
   if (st != MLP_OK) return st;
   return fc2_forward(s, H, fc2_lo(mode, H_lo), B, b, Y, ws, L);
@@ -943,8 +1198,9 @@ mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A, const
   st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {B, "B", false}, {Z, "Z", false, s.T == 0},
                     {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
                     {dB, "dB", false}, {db, "db", true}},
-                ws, ws_bytes, stream, L);
+                ws, ws_bytes, stream, L, false, mode);
   if (st != MLP_OK) return st;
+  if (mode == MLP_TP_FP8) return backward_fp8(s, dY, X, A, B, Z, H, H_lo, dX, dA, da, dB, db, ws, false, L);
   void* dH = static_cast<char*>(ws) + dh_offset();
   void* dH_lo = static_cast<char*>(ws) + dh_lo_offset(s);
   if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
@@ -970,12 +1226,13 @@ mlp_status_t mlp_tp_forward_recompute(const void* X, const void* A, const void* 
   if (st != MLP_OK) return st;
   st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {B, "B", false}, {b, "b", false},
                     {Y, "Y", false, s.T == 0}},
-                ws, ws_bytes, stream, L, true);
+                ws, ws_bytes, stream, L, true, mode);
   if (st != MLP_OK) return st;
   char* w = static_cast<char*>(ws);
   void* Z = w + recompute_z_offset(s);
   void* H = w + recompute_h_offset(s);
   void* H_lo = w + recompute_hlo_offset(s);
+  if (mode == MLP_TP_FP8) return forward_fp8(s, X, A, a, B, b, Y, Z, H, H_lo, ws, true, L);
   if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
   return fc2_forward(s, H, fc2_lo(mode, H_lo), B, b, Y, ws, L);
 }
@@ -990,7 +1247,7 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
   st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false},
                     {B, "B", false}, {dX, "dX", false, s.T == 0}, {dA, "dA", false}, {da, "da", true},
                     {dB, "dB", false}, {db, "db", true}},
-                ws, ws_bytes, stream, L, true);
+                ws, ws_bytes, stream, L, true, mode);
   if (st != MLP_OK) return st;
   char* w = static_cast<char*>(ws);
   void* Z = w + recompute_z_offset(s);
@@ -999,11 +1256,119 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
   void* dH = w + dh_offset();
   void* dH_lo = w + dh_lo_offset(s);
   // recompute the activations the forward did not keep, then the backward
+  if (mode == MLP_TP_FP8) {
+    if ((st = fc1_forward_fp8(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
+    return backward_fp8(s, dY, X, A, B, Z, H, H_lo, dX, dA, da, dB, db, ws, true, L);
+  }
   if ((st = fc1_forward(s, X, A, a, Z, H, H_lo, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_data(s, dY, B, Z, dH, dH_lo, da, ws, L)) != MLP_OK) return st;
   if ((st = fc2_backward_weight(s, H, H_lo, dY, dB, db, ws, L)) != MLP_OK) return st;
   if ((st = fc1_backward_data(s, dH, fc1_bwd_lo(mode, dH_lo), A, dX, ws, L)) != MLP_OK) return st;
   return fc1_backward_weight(s, X, dH, dH_lo, dA, ws, L);
+}
+
+size_t mlp_tp_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode) {
+  Shape s{T, h, f, t};
+  std::string saved = g_last_error;
+  const bool ok = check_shape(s) == MLP_OK && check_mode(mode) == MLP_OK;
+  g_last_error = saved;
+  return ok ? mode_workspace_bytes(s, mode, false) : 0;
+}
+
+size_t mlp_tp_recompute_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode) {
+  Shape s{T, h, f, t};
+  std::string saved = g_last_error;
+  const bool ok = check_shape(s) == MLP_OK && check_mode(mode) == MLP_OK;
+  g_last_error = saved;
+  return ok ? mode_workspace_bytes(s, mode, true) : 0;
+}
+
+// ---- the fp16 + e4m3 mode, stage by stage
+mlp_status_t mlp_tp_fp8_prepare_forward(const void* B, int64_t T, int64_t h, int64_t f, int32_t t, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{B, "B", false}}, ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fp8_prepare_forward(s, B, fp8_bufs(ws, s, false), ws, L);
+}
+
+mlp_status_t mlp_tp_fp8_prepare_backward(const void* dY, const void* X, const void* A, const void* B, int64_t T,
+                                         int64_t h, int64_t f, int32_t t, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{dY, "dY", false, s.T == 0}, {X, "X", false, s.T == 0}, {A, "A", false}, {B, "B", false}},
+                             ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fp8_prepare_backward(s, dY, X, A, B, fp8_bufs(ws, s, false), ws, L);
+}
+
+mlp_status_t mlp_tp_fc1_forward_fp8(const void* X, const void* A, const void* a, int64_t T, int64_t h, int64_t f,
+                                    int32_t t, void* Z, void* H, void* H_lo, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{X, "X", false, s.T == 0}, {A, "A", false}, {a, "a", false}, {Z, "Z", false, s.T == 0},
+                                 {H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}},
+                             ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fc1_forward_fp8(s, X, A, a, Z, H, H_lo, ws, L);
+}
+
+mlp_status_t mlp_tp_fc2_forward_fp8(const void* H, const void* b, int64_t T, int64_t h, int64_t f, int32_t t, void* Y,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{H, "H", false, s.T == 0}, {b, "b", true}, {Y, "Y", false, s.T == 0}}, ws, ws_bytes,
+                             stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fc2_forward_fp8(s, H, fp8_bufs(ws, s, false).w16, b, Y, ws, L);
+}
+
+mlp_status_t mlp_tp_fc2_backward_data_fp8(const void* dY, const void* B, const void* Z, int64_t T, int64_t h,
+                                          int64_t f, int32_t t, void* dH, void* dH_lo, void* da, void* ws,
+                                          size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{dY, "dY", false, s.T == 0}, {B, "B", false}, {Z, "Z", false, s.T == 0},
+                                 {dH, "dH", false, s.T == 0}, {dH_lo, "dH_lo", false, s.T == 0}, {da, "da", true}},
+                             ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fc2_backward_data_fp8(s, dY, B, Z, dH, dH_lo, da, fp8_bufs(ws, s, false).stats, ws, L);
+}
+
+mlp_status_t mlp_tp_fc2_backward_weight_fp8(const void* H, const void* H_lo, const void* dY, int64_t T, int64_t h,
+                                            int64_t f, int32_t t, void* dB, void* db, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{H, "H", false, s.T == 0}, {H_lo, "H_lo", false, s.T == 0}, {dY, "dY", false, s.T == 0},
+                                 {dB, "dB", false}, {db, "db", true}},
+                             ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  const Fp8Bufs q = fp8_bufs(ws, s, false);
+  return fc2_backward_weight_fp8(s, H, H_lo, q.dy16, q.dy8, dY, dB, db, q.stats, ws, L);
+}
+
+mlp_status_t mlp_tp_fc1_backward_data_fp8(const void* dH, int64_t T, int64_t h, int64_t f, int32_t t, void* dX,
+                                          void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{dH, "dH", false, s.T == 0}, {dX, "dX", false, s.T == 0}}, ws, ws_bytes, stream, L,
+                             false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  const Fp8Bufs q = fp8_bufs(ws, s, false);
+  return fc1_backward_data_fp8(s, dH, q.w16, dX, q.stats, ws, L);
+}
+
+mlp_status_t mlp_tp_fc1_backward_weight_fp8(const void* dH, const void* dH_lo, int64_t T, int64_t h, int64_t f,
+                                            int32_t t, void* dA, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, f, t};
+  Launch L;
+  mlp_status_t st = prologue(s, {{dH, "dH", false, s.T == 0}, {dH_lo, "dH_lo", false, s.T == 0}, {dA, "dA", false}},
+                             ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  const Fp8Bufs q = fp8_bufs(ws, s, false);
+  return fc1_backward_weight_fp8(s, q.x16, q.x8, dH, dH_lo, dA, q.stats, ws, L);
 }
 
 mlp_status_t mlp_tp_check(void* ws, void* stream) {
@@ -1023,6 +1388,7 @@ const char* mlp_tp_status_string(mlp_status_t status) {
     case MLP_ERR_CUDA: return "MLP_ERR_CUDA";
     case MLP_ERR_BOUNDS: return "MLP_ERR_BOUNDS";
     case MLP_ERR_TIMEOUT: return "MLP_ERR_TIMEOUT";
+    case MLP_ERR_RANGE: return "MLP_ERR_RANGE";
   }
   return "MLP_ERR_UNKNOWN";
 }

@@ -113,8 +113,44 @@ def test_binding_refuses_cpu_tensors(lib):
         binding.mlp_tp_fc1_forward(x, x, x, 64, 256, 1024, 2, x, x, x, (FAKE, 1 << 30), stream=0)
 
 
+def test_fp8_workspace_bytes(lib):
+    """MLP_TP_FP8 adds its operand copies after the mode-independent
+    workspace: W16 (fp16 B or A, 2·h·f), X16 and dY16 (2·T·h each), X8 and
+    dY8 (T·h each), each rounded up to 256 bytes."""
+    T, h, f, t = 200, 192, 384, 6
+    rnd = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    extra = rnd(2 * h * f) + 2 * rnd(2 * T * h) + 2 * rnd(T * h)
+    for mode in (binding.ACCURATE, binding.FAST_FC2_FORWARD, binding.FAST):
+        assert binding.workspace_bytes_mode(T, h, f, t, mode) == binding.workspace_bytes(T, h, f, t)
+        assert binding.recompute_workspace_bytes_mode(T, h, f, t, mode) == binding.recompute_workspace_bytes(T, h, f, t)
+    assert binding.workspace_bytes_mode(T, h, f, t, binding.FP8) == binding.workspace_bytes(T, h, f, t) + extra
+    assert (binding.recompute_workspace_bytes_mode(T, h, f, t, binding.FP8)
+            == binding.recompute_workspace_bytes(T, h, f, t) + extra)
+    assert binding.workspace_bytes_mode(T, h, f, t, 5) == 0
+    assert binding.workspace_bytes_mode(T, h, 100, t, binding.FP8) == 0
+
+
+def test_fp8_mode_checks_its_workspace(lib):
+    T, h, f, t = 64, 256, 1024, 2
+    small = binding.workspace_bytes(T, h, f, t)  # enough for every other mode
+    st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, T, h, f, t, binding.FP8, FAKE, FAKE, FAKE, FAKE,
+                            FAKE * 2, small, None)
+    assert st == 4 and "workspace" in binding.mlp_tp_last_error()
+    st = lib.mlp_tp_fc2_backward_weight_fp8(FAKE, FAKE, FAKE, T, h, f, t, FAKE, None, FAKE * 2, small, None)
+    assert st == 4
+    # with enough workspace the call gets as far as the device check (no GPU
+    # here; with one, fake addresses must never reach a launch)
+    import torch
+    if torch.cuda.is_available():
+        return
+    big = binding.workspace_bytes_mode(T, h, f, t, binding.FP8)
+    st = lib.mlp_tp_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, T, h, f, t, binding.FP8, FAKE, FAKE, None,
+                             FAKE, None, FAKE * 2, big, None)
+    assert st == 5
+
+
 def test_precision_mode_is_validated(lib):
-    for bad in (4, 7, -1):
+    for bad in (5, 7, -1):
         st = lib.mlp_tp_forward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, 1024, 2, bad, FAKE, FAKE, FAKE, FAKE,
                                 FAKE * 2, 1 << 30, None)
         assert st == 1 and "precision mode" in binding.mlp_tp_last_error()
