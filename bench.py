@@ -124,6 +124,74 @@ def roofline_entry(stage_ms, mode, T, h, f, clocks, peaks, peak_src):
             "stage_clocks": clocks}
 
 
+FP8_STAGES = ("fp8_prepare_forward", "fc1_forward", "fc2_forward", "fp8_prepare_backward", "fc2_backward_data",
+              "fc2_backward_weight", "fc1_backward_data", "fc1_backward_weight")
+# tensor time of each stage's GEMM in bf16-product units (an e4m3 product of K = 32 takes the time of a
+# bf16 product of K = 16)
+FP8_STAGE_PRODUCTS = {"fc1_forward": 1, "fc2_forward": 1, "fc2_backward_data": 1, "fc2_backward_weight": 1.5,
+                      "fc1_backward_data": 1, "fc1_backward_weight": 1.5}
+
+
+def fp8_leg(binding, dev, T, h, f, t, steps, stream, clock_interval_ms, local, check_every=None):
+    """The fp16 + e4m3 mode (MLP_TP_FP8) through its stage calls: the whole
+    step timed by events around `steps` steps, then the stages by events
+    between the calls, with the clocks of each window."""
+    import torch
+    sh = stream.cuda_stream
+    e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
+    Z = torch.empty(T, f, dtype=torch.float32, device="cuda")
+    H16, dH16 = (torch.empty(T, f, dtype=torch.float16, device="cuda") for _ in range(2))
+    H8, dH8 = (torch.empty(T, f, dtype=torch.uint8, device="cuda") for _ in range(2))
+    Y, dX, dA, dB, da, db = e(T, h), e(T, h), e(h, f), e(f, h), e(f), e(h)
+    ws = binding.make_workspace_mode(T, h, f, t, binding.FP8)
+    calls = (
+        lambda: binding.mlp_tp_fp8_prepare_forward(dev["B"], T, h, f, t, ws, sh),
+        lambda: binding.mlp_tp_fc1_forward_fp8(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H16, H8, ws, sh),
+        lambda: binding.mlp_tp_fc2_forward_fp8(H16, dev["b"], T, h, f, t, Y, ws, sh),
+        lambda: binding.mlp_tp_fp8_prepare_backward(dev["dY"], dev["X"], dev["A"], dev["B"], T, h, f, t, ws, sh),
+        lambda: binding.mlp_tp_fc2_backward_data_fp8(dev["dY"], dev["B"], Z, T, h, f, t, dH16, dH8, da, ws, sh),
+        lambda: binding.mlp_tp_fc2_backward_weight_fp8(H16, H8, dev["dY"], T, h, f, t, dB, db, ws, sh),
+        lambda: binding.mlp_tp_fc1_backward_data_fp8(dH16, T, h, f, t, dX, ws, sh),
+        lambda: binding.mlp_tp_fc1_backward_weight_fp8(dH16, dH8, T, h, f, t, dA, ws, sh),
+    )
+
+    def step(evs=None):
+        for i, c in enumerate(calls):
+            if evs is not None:
+                evs[i].record(stream)
+            c()
+        if evs is not None:
+            evs[len(calls)].record(stream)
+
+    for _ in range(3):
+        step()
+    binding.mlp_tp_check(ws, sh)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local, clock_interval_ms) as clk:
+        l0 = binding.mlp_tp_launch_count()
+        s0.record(stream)
+        for _ in range(steps):
+            step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        launches = binding.mlp_tp_launch_count() - l0
+    binding.mlp_tp_check(ws, sh)
+    ms = s0.elapsed_time(s1)
+    n_ev = max(10, steps // 4)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n_ev)]
+    torch.cuda.synchronize()
+    with ClockSampler(local, clock_interval_ms) as clk_st:
+        for k in range(n_ev):
+            step(ev[k])
+        torch.cuda.synchronize()
+    binding.mlp_tp_check(ws, sh)
+    stage_ms = {s: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(n_ev))
+                for i, s in enumerate(FP8_STAGES)}
+    return {"ms": ms, "steps": steps, "launches": launches, "clocks": clk.summary(), "stage_ms": stage_ms,
+            "stage_clocks": clk_st.summary()}
+
+
 # ---------------------------------------------------------------- helpers
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -347,6 +415,7 @@ def main():
     ap.add_argument("--no-peer", action="store_true", help="skip the one-GPU leg of the cross-GPU reduction path")
     ap.add_argument("--stage-steps", type=int, default=None,
                     help="steps of the per-stage timing pass (default: enough for 0.3 s; small for ncu captures)")
+    ap.add_argument("--no-fp8-leg", action="store_true", help="skip timing the fp16 + e4m3 mode")
     ap.add_argument("--no-accurate-leg", action="store_true",
                     help="with the fast mode timed, skip timing the accurate mode beside it")
     ap.add_argument("--clock-interval-ms", type=int, default=50,
@@ -478,6 +547,29 @@ def main():
                     "steps": args.steps, "clocks": clk_a,
                     "api": "the same stage calls with the low half of the pair in the Y and dX GEMMs "
                            "(the library's default mode)"}
+
+    # ------------------------------------------------ the fp16 + e4m3 mode (MLP_TP_FP8) beside them
+    fp8 = None
+    if not args.no_fp8_leg and world == 1:
+        r8 = fp8_leg(binding, dev, T, h, f, t, args.steps, stream, args.clock_interval_ms, local)
+        peaks8, src8 = load_peaks()
+        gemm_stages = [k for k in r8["stage_ms"] if k in FP8_STAGE_PRODUCTS]
+        dom = max(gemm_stages, key=lambda k: r8["stage_ms"][k])
+        unit = 2.0 * T * h * f
+        ach = unit / (r8["stage_ms"][dom] * 1e-3) / 1e12
+        ck = r8["stage_clocks"]
+        settled = bool(ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] < 0.97 * ck["sm_max_mhz"])
+        pk = float(peaks8.get("bf16_tflops_sustained" if settled else "bf16_tflops",
+                              FALLBACK_PEAKS["bf16_tflops_sustained" if settled else "bf16_tflops"]))
+        fp8 = {"value": float(wl.flops) * r8["steps"] / (r8["ms"] * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": r8["ms"] / r8["steps"], "steps": r8["steps"], "gpu_launches": r8["launches"],
+               "clocks": r8["clocks"], "stage_ms": r8["stage_ms"],
+               "tensor_units_per_step": sum(FP8_STAGE_PRODUCTS.values()),
+               "dominant": {"stage": dom, "achieved": ach, "peak": pk, "frac": ach / pk,
+                            "peak_source": src8 + (" bf16_tflops_sustained" if settled else " bf16_tflops (burst)"),
+                            "executed_tflops": ach * FP8_STAGE_PRODUCTS[dom], "stage_clocks": ck},
+               "api": "mlp_tp_fp8_prepare_forward, the two forward stages, mlp_tp_fp8_prepare_backward and the "
+                      "four backward stages of MLP_TP_FP8 (fp16 operands, e4m3 residual products in dA, dB)"}
 
     # ------------------------------------------------ steady state: the same loop for >= 2 s
     steady = None
@@ -775,6 +867,8 @@ def main():
     }
     if accurate is not None:
         line["accurate"] = accurate
+    if fp8 is not None:
+        line["fp8"] = fp8
     if steady is not None:
         line["steady"] = steady
     if peer is not None:

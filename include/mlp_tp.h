@@ -144,7 +144,10 @@ typedef enum {
  * formats cannot hold (|H| >= 2^13; a weight beyond 65504) are reported as
  * MLP_ERR_RANGE by mlp_tp_check.  Every output stays within
  * 1e-2·(|exact| + 1) of the exact block on all five workloads the tests run,
- * the 8.3B-class one included.  This mode needs
+ * the 8.3B-class one included.  Y and dX carry 11 bits of H and dH: with
+ * pre-activations near 40 and weights ~N(0, 0.3) (a stress case, not a
+ * workload) Y reaches 1.96x the tolerance, where MLP_TP_ACCURATE keeps 16
+ * bits.  This mode needs
  * mlp_tp_workspace_bytes_mode(..., MLP_TP_FP8) bytes of workspace (the
  * copies X16, X8, dY16, dY8 and fp16 B or A: 6·T·h + 2·h·f more bytes). */
 size_t mlp_tp_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode);
