@@ -375,6 +375,18 @@ mlp_status_t mlp_tp_fc1_backward_data_peer(const void* dH, const void* dH_lo, co
                                            int64_t T, int64_t h, int64_t fs, const mlp_tp_peer_t* peer,
                                            void* ws, size_t ws_bytes, void* stream);
 
+/* The same two GEMMs in MLP_TP_FP8 form, after mlp_tp_fp8_prepare_forward /
+ * mlp_tp_fp8_prepare_backward on this rank's shard (t = 1, f = fs) and
+ * workspace (mlp_tp_workspace_bytes_mode(T, h, fs, 1, MLP_TP_FP8) bytes):
+ * P_r = H16·fp16(B_r) and Q_r = dH16·fp16(A_r)ᵀ / sH with H, dH fp16 [T, fs].
+ * Each rank's sH follows from its own shard of B; the fp32 partials carry no
+ * scale, so the owner's sum is the same call as in the other modes. */
+mlp_status_t mlp_tp_fc2_forward_peer_fp8(const void* H, int64_t T, int64_t h, int64_t fs,
+                                         const mlp_tp_peer_t* peer, void* ws, size_t ws_bytes, void* stream);
+mlp_status_t mlp_tp_fc1_backward_data_peer_fp8(const void* dH, int64_t T, int64_t h, int64_t fs,
+                                               const mlp_tp_peer_t* peer, void* ws, size_t ws_bytes,
+                                               void* stream);
+
 /* The owner's sum: out[T/world, h] = bf16(Σ_r slot r + bias), rank order.
  * `ws` needs only its 256-byte status header here. */
 mlp_status_t mlp_tp_peer_reduce(const mlp_tp_peer_t* peer, const void* bias, int64_t T, int64_t h,

@@ -76,6 +76,8 @@ _SIGS = {
     "mlp_tp_peer_flag_bytes": ([_I64, _I64, _I32], _SZ),
     "mlp_tp_fc2_forward_peer": ([_P] * 3 + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_fc1_backward_data_peer": ([_P] * 3 + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc2_forward_peer_fp8": ([_P] + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
+    "mlp_tp_fc1_backward_data_peer_fp8": ([_P] + [_I64] * 3 + [_PP] + [_P, _SZ, _P], ctypes.c_int),
     "mlp_tp_peer_reduce": ([_PP, _P, _I64, _I64, _P, _P, _SZ, _P], ctypes.c_int),
     "mlp_tp_ipc_export": ([_P, _P, ctypes.POINTER(ctypes.c_uint64)], ctypes.c_int),
     "mlp_tp_ipc_import": ([_P, ctypes.c_uint64, ctypes.POINTER(_P)], ctypes.c_int),
@@ -386,6 +388,18 @@ def mlp_tp_fc1_backward_data_peer(dH, dH_lo, A, T, h, fs, peer: Peer, ws, stream
     w, wn = _ws(ws)
     _check(lib().mlp_tp_fc1_backward_data_peer(_addr(dH, "dH", T == 0), _addr(dH_lo, "dH_lo", True), _addr(A, "A"),
                                                T, h, fs, ctypes.byref(peer), w, wn, _stream(stream)))
+
+
+def mlp_tp_fc2_forward_peer_fp8(H, T, h, fs, peer: Peer, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc2_forward_peer_fp8(_addr(H, "H", T == 0, "f16"), T, h, fs, ctypes.byref(peer), w, wn,
+                                             _stream(stream)))
+
+
+def mlp_tp_fc1_backward_data_peer_fp8(dH, T, h, fs, peer: Peer, ws, stream=None):
+    w, wn = _ws(ws)
+    _check(lib().mlp_tp_fc1_backward_data_peer_fp8(_addr(dH, "dH", T == 0, "f16"), T, h, fs, ctypes.byref(peer),
+                                                   w, wn, _stream(stream)))
 
 
 def mlp_tp_peer_reduce(peer: Peer, bias, T, h, out, ws, stream=None):

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(STATS_THREADS) fp8_stats_kernel(const __nv_bfl
     const long long row = which == 0 ? r : (which == 1 ? r - T : r - 2LL * T);
     const __nv_bfloat16* src = (which == 0 ? X : (which == 1 ? dY : B)) + row * h;
     float mx = 0.0f, ss = 0.0f;
+#pragma unroll 4
     for (int c = lane * 8; c < h; c += 256) {
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + c));
       const uint32_t u[4] = {w.x, w.y, w.z, w.w};
@@ -199,31 +200,49 @@ struct CastJobs {
   int count;
 };
 
+constexpr int CAST_UNROLL = 4;  // 16-byte loads in flight per thread
+
+__device__ __forceinline__ void cast_group(const uint4 w, const CastJob& jb, float s, float s8, long long g,
+                                           bool& bad) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o16[4], o8[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+    if (jb.scale == CAST_UNSCALED) bad |= fabsf(v.x) > FP16_MAX || fabsf(v.y) > FP16_MAX;
+    o16[e] = pack_f16x2(v.x * s, v.y * s);
+    o8[e >> 1] |= pack_e4m3x2(v.x * s8, v.y * s8) << (16 * (e & 1));
+  }
+  reinterpret_cast<uint4*>(jb.dst16)[g] = make_uint4(o16[0], o16[1], o16[2], o16[3]);
+  if (jb.dst8 != nullptr) reinterpret_cast<uint2*>(jb.dst8)[g] = make_uint2(o8[0], o8[1]);
+}
+
 __global__ void __launch_bounds__(256) fp8_cast_kernel(const __grid_constant__ CastJobs jobs, const unsigned int* stats,
                                                        unsigned int* status) {
   grid_wait_prerequisites();
   grid_launch_dependents();
   const Fp8Scales sc = stats != nullptr ? fp8_scales(stats) : Fp8Scales{1.0f, 1.0f, 1.0f};
   bool bad = false;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (int j = 0; j < jobs.count; ++j) {
     const CastJob& jb = jobs.job[j];
     const float s = jb.scale == CAST_SX ? sc.sX : (jb.scale == CAST_SY ? sc.sY : 1.0f);
     const float s8 = s / FP8_LO_SHIFT;
-    const long long groups = jb.n / 8;
-    for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
-         g += static_cast<long long>(gridDim.x) * blockDim.x) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(jb.src) + g);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-      uint32_t o16[4], o8[2] = {0u, 0u};
+    const long long groups = jb.n / 8;  // 8 values (16 bytes of bf16) per group
+    const uint4* src = reinterpret_cast<const uint4*>(jb.src);
+    for (long long g0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g0 < groups;
+         g0 += CAST_UNROLL * stride) {
+      uint4 w[CAST_UNROLL];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
-        if (jb.scale == CAST_UNSCALED) bad |= fabsf(v.x) > FP16_MAX || fabsf(v.y) > FP16_MAX;
-        o16[e] = pack_f16x2(v.x * s, v.y * s);
-        o8[e >> 1] |= pack_e4m3x2(v.x * s8, v.y * s8) << (16 * (e & 1));
+      for (int q = 0; q < CAST_UNROLL; ++q) {
+        const long long g = g0 + q * stride;
+        w[q] = g < groups ? __ldg(src + g) : make_uint4(0u, 0u, 0u, 0u);
       }
-      reinterpret_cast<uint4*>(jb.dst16)[g] = make_uint4(o16[0], o16[1], o16[2], o16[3]);
-      if (jb.dst8 != nullptr) reinterpret_cast<uint2*>(jb.dst8)[g] = make_uint2(o8[0], o8[1]);
+#pragma unroll
+      for (int q = 0; q < CAST_UNROLL; ++q) {
+        const long long g = g0 + q * stride;
+        if (g < groups) cast_group(w[q], jb, s, s8, g, bad);
+      }
     }
   }
   if (bad) {

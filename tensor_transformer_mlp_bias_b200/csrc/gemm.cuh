@@ -838,18 +838,18 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(r[j]) + bias[j];
             if (p.fp8_out) {
               // H as fp16 plus its e4m3 residual (H − fp16(H))·2^7
-              bool big = false;
+              float big = 0.0f;  // max |H| of the chunk
 #pragma unroll
               for (int j = 0; j < 8; ++j) lp[j] = 0u;
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const float g0 = gelu_f(z[2 * j]), g1 = gelu_f(z[2 * j + 1]);
-                big |= fabsf(g0) >= FP8_H_LIMIT || fabsf(g1) >= FP8_H_LIMIT;
+                big = fmaxf(big, fmaxf(fabsf(g0), fabsf(g1)));
                 uint32_t lo8;
                 split_f16_e4m3(g0, g1, hp[j], lo8);
                 lp[j >> 1] |= lo8 << (16 * (j & 1));
               }
-              record_range(p, big, 0xB01u);
+              record_range(p, big >= FP8_H_LIMIT, 0xB01u);
               stage_f32x32(st_f32, lane, z);
               stage_bf16x32(st_out0, lane, hp);  // fp16: same 64-byte rows and swizzle
               stage_e4m3x32(st_out1, lane, reinterpret_cast<const uint32_t(&)[8]>(lp));
@@ -878,18 +878,18 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             uint32_t hp[16], lp[16];
             if (p.fp8_out) {
               // dH·sH as fp16 plus its e4m3 residual
-              bool big = false;
+              float big = 0.0f;  // max |dH·sH| of the chunk
 #pragma unroll
               for (int j = 0; j < 8; ++j) lp[j] = 0u;
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const float d0 = dh[2 * j] * s_dh, d1 = dh[2 * j + 1] * s_dh;
-                big |= fabsf(d0) >= FP8_H_LIMIT || fabsf(d1) >= FP8_H_LIMIT;
+                big = fmaxf(big, fmaxf(fabsf(d0), fabsf(d1)));
                 uint32_t lo8;
                 split_f16_e4m3(d0, d1, hp[j], lo8);
                 lp[j >> 1] |= lo8 << (16 * (j & 1));
               }
-              record_range(p, big, 0xB02u);
+              record_range(p, big >= FP8_H_LIMIT, 0xB02u);
               stage_bf16x32(st_out0, lane, hp);
               stage_e4m3x32(st_out1, lane, reinterpret_cast<const uint32_t(&)[8]>(lp));
             } else {
@@ -917,7 +917,7 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
             if (peer_blk) {
               float v[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * out_mul;  // 1 outside the fp8 mode
               stage_f32x32(st_f32, lane, v);
               __syncwarp();
               const long long base =
@@ -979,19 +979,22 @@ __global__ void __launch_bounds__(TileCfg<PAIR, TN, EPI, EW, DUAL>::THREADS, 1)
                                       sum[c * 32 + 4 * j + 3]);
               }
             } else if (s == it.s_end - 1) {
-              float bias[32];
-              if (p.bias != nullptr) {
-                load_bf16x32(p.bias + col, bias);
-              } else {
+              // 8 columns at a time (one 16-byte bias load, one 16-byte
+              // staging store), so few values beyond the running sums are live
 #pragma unroll
-                for (int j = 0; j < 32; ++j) bias[j] = 0.0f;
+              for (int g = 0; g < 4; ++g) {
+                const uint4 braw = p.bias != nullptr ? __ldg(reinterpret_cast<const uint4*>(p.bias + col) + g)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+                uint32_t yp[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 bv = unpack_bf16x2(bw[e]);
+                  yp[e] = pack_bf16x2(fmaf(sum[c * 32 + 8 * g + 2 * e], out_mul, bv.x),
+                                      fmaf(sum[c * 32 + 8 * g + 2 * e + 1], out_mul, bv.y));
+                }
+                st_shared_v4(st_out0 + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4), yp[0], yp[1], yp[2], yp[3]);
               }
-              uint32_t yp[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                yp[j] = pack_bf16x2(fmaf(sum[c * 32 + 2 * j], out_mul, bias[2 * j]),
-                                    fmaf(sum[c * 32 + 2 * j + 1], out_mul, bias[2 * j + 1]));
-              stage_bf16x32(st_out0, lane, yp);
               fence_proxy_async_shared();
               __syncwarp();
               if (lane == 0) {

@@ -858,6 +858,11 @@ Operand op16(const void* p, bool mn) { return Operand{{p, p}, mn, {OP_F16, OP_F1
 Operand op16_8(const void* p16, const void* p8, bool mn) { return Operand{{p16, p8}, mn, {OP_F16, OP_E4M3}}; }
 
 // Z = X·A + a (fp32), H16 = fp16(g(Z)), H8 = e4m3((g(Z) − H16)·2^7).
+// Always 256-column tiles: two accumulators let the epilogue (whose fp16 +
+// e4m3 split costs more arithmetic than the bf16 pair) overlap the next
+// tile's mainloop.  Measured on B200 against 512-column tiles: 0.526 vs
+// 0.551 ms at T=4096, h=4096, f=16384; 1.25 vs 1.39 ms at T=16384, h=3072,
+// f=12288; equal at T=8192, h=1024, f=4096.
 mlp_status_t fc1_forward_fp8(const Shape& s, const void* X, const void* A, const void* a, void* Z, void* H16,
                              void* H8, void* ws, const Launch& L) {
   GemmParams p = base_params(ws);
@@ -867,18 +872,6 @@ mlp_status_t fc1_forward_fp8(const Shape& s, const void* X, const void* A, const
   p.bias = static_cast<const __nv_bfloat16*>(a);
   p.fp8_out = 1;
   GemmDesc g{one(X, false), one(A, true), s.T, s.f, s.h, 1, 1};
-  if (kFc1TN == 512) {
-    const int pairs = L.sms / TileShape::CTAS;
-    const int64_t mt = (s.T + TileShape::TILE_M - 1) / TileShape::TILE_M;
-    auto wave_eff = [&](int64_t tn) {
-      const int64_t tiles = mt * ((s.f + tn - 1) / tn);
-      const int64_t waves = (tiles + pairs - 1) / pairs;
-      return static_cast<double>(tiles) / static_cast<double>(waves * pairs);
-    };
-    const int64_t tiles256 = mt * ((s.f + 255) / 256);
-    if (tiles256 > pairs && wave_eff(512) + 0.05 >= wave_eff(256))
-      return launch_gemm<false, true, EPI_BIAS_GELU, kFc1TN>(g, p, L, "column-parallel forward (Z, H16, H8)");
-  }
   return launch_gemm<false, true, EPI_BIAS_GELU, 256>(g, p, L, "column-parallel forward (Z, H16, H8)");
 }
 
@@ -1063,6 +1056,31 @@ mlp_status_t fc1_backward_data_peer(const Shape& s, const void* dH, const void* 
     return launch_gemm<false, false, EPI_PEER, 256, kPair, 8, kDualA>(g, p, L,
                                                                      "column-parallel backward data to the owners (Q)");
   return launch_gemm<false, false, EPI_PEER>(g, p, L, "column-parallel backward data to the owners (Q)");
+}
+
+// The fp16 + e4m3 mode's row-parallel GEMMs of one rank: H16·B16 (B16 from
+// the workspace) and dH16·A16ᵀ / sH (A16 and the statistics from the
+// workspace), fp32 partials to the owners.
+mlp_status_t fc2_forward_peer_fp8(const Shape& s, const void* H16, const void* B16, const PeerParams& q,
+                                  long long recv_elems, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.peer = q;
+  p.peer_recv_elems = recv_elems;
+  p.f16_ops = 1;
+  GemmDesc g{op16(H16, false), op16(B16, true), s.T, s.h, s.f, 1, 1};
+  return launch_gemm<false, true, EPI_PEER>(g, p, L, "row-parallel forward to the owners (P, fp16)");
+}
+
+mlp_status_t fc1_backward_data_peer_fp8(const Shape& s, const void* dH16, const void* A16, const unsigned int* stats,
+                                        const PeerParams& q, long long recv_elems, void* ws, const Launch& L) {
+  GemmParams p = base_params(ws);
+  p.peer = q;
+  p.peer_recv_elems = recv_elems;
+  p.f16_ops = 1;
+  p.fp8_stats = stats;
+  p.out_scale = OUT_SCALE_INV_SH;
+  GemmDesc g{op16(dH16, false), op16(A16, false), s.T, s.h, s.f, 1, 1};
+  return launch_gemm<false, false, EPI_PEER>(g, p, L, "column-parallel backward data to the owners (Q, fp16)");
 }
 
 // Common preamble: shape, pointers, workspace, device.
@@ -1437,6 +1455,33 @@ mlp_status_t mlp_tp_fc1_backward_data_peer(const void* dH, const void* dH_lo, co
                 stream, L);
   if (st != MLP_OK) return st;
   return fc1_backward_data_peer(s, dH, dH_lo, A, q, recv_elems, ws, L);
+}
+
+mlp_status_t mlp_tp_fc2_forward_peer_fp8(const void* H, int64_t T, int64_t h, int64_t fs, const mlp_tp_peer_t* peer,
+                                         void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, fs, 1};
+  Launch L;
+  PeerParams q;
+  long long recv_elems = 0;
+  mlp_status_t st = check_shape(s);
+  if (st != MLP_OK || (st = check_peer(peer, T, h, q, recv_elems)) != MLP_OK) return st;
+  st = prologue(s, {{H, "H", false, s.T == 0}}, ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  return fc2_forward_peer_fp8(s, H, fp8_bufs(ws, s, false).w16, q, recv_elems, ws, L);
+}
+
+mlp_status_t mlp_tp_fc1_backward_data_peer_fp8(const void* dH, int64_t T, int64_t h, int64_t fs,
+                                               const mlp_tp_peer_t* peer, void* ws, size_t ws_bytes, void* stream) {
+  Shape s{T, h, fs, 1};
+  Launch L;
+  PeerParams q;
+  long long recv_elems = 0;
+  mlp_status_t st = check_shape(s);
+  if (st != MLP_OK || (st = check_peer(peer, T, h, q, recv_elems)) != MLP_OK) return st;
+  st = prologue(s, {{dH, "dH", false, s.T == 0}}, ws, ws_bytes, stream, L, false, MLP_TP_FP8);
+  if (st != MLP_OK) return st;
+  const Fp8Bufs b = fp8_bufs(ws, s, false);
+  return fc1_backward_data_peer_fp8(s, dH, b.w16, b.stats, q, recv_elems, ws, L);
 }
 
 mlp_status_t mlp_tp_peer_reduce(const mlp_tp_peer_t* peer, const void* bias, int64_t T, int64_t h, void* out,

@@ -35,6 +35,12 @@ dY arrive split by tokens (rank r holds rows [r·T/N, (r+1)·T/N)).  They are
 all-gathered before the GEMMs, and Y and dX stay split by tokens: the
 reduce-scatter alone.
 
+Precision modes: as the composite calls (mode=binding.ACCURATE by default).
+With binding.FP8 each rank runs the fp16 + e4m3 stage calls on its shard: the
+prepare calls cast its B_i (forward) and X, dY, A_i (backward) in its own
+workspace, and the row-parallel GEMMs send unscaled fp32 partials (each rank
+undoes its own dH scale), so the reduction is the same in every mode.
+
 `ops` is the object whose stage calls run the GEMMs: the C-ABI binding,
 unless a caller supplies another implementation with the same signatures.
 """
@@ -142,6 +148,11 @@ def _dtypes(ops) -> Tuple[torch.dtype, torch.dtype]:
     return getattr(ops, "DTYPE", torch.bfloat16), getattr(ops, "Z_DTYPE", torch.float32)
 
 
+def _fp8_dtypes(ops) -> Tuple[torch.dtype, torch.dtype]:
+    """Element types of the fp16 + e4m3 mode's activations (fp16 value, e4m3 residual)."""
+    return getattr(ops, "F16_DTYPE", torch.float16), getattr(ops, "E4M3_DTYPE", torch.uint8)
+
+
 def _gather_tokens(x: torch.Tensor, group) -> torch.Tensor:
     world = dist.get_world_size(group)
     out = torch.empty(x.shape[0] * world, *x.shape[1:], dtype=x.dtype, device=x.device)
@@ -196,15 +207,25 @@ def forward(X: torch.Tensor, A_i: torch.Tensor, a_i: torch.Tensor, B_i: torch.Te
     owns = reduction == "peer" and exchange is None
     if owns:
         exchange = PeerExchange(T, h, group, dev, ops)
-    ws = ops.make_workspace(T, h, fs, 1, dev)
     Z = torch.empty(T, fs, dtype=zdt, device=dev)
-    H = torch.empty(T, fs, dtype=dt, device=dev)
-    H_lo = torch.empty(T, fs, dtype=dt, device=dev)
-    ops.mlp_tp_fc1_forward(X, A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws)
-    lo = None if mode & binding.FAST_FC2_FORWARD else H_lo
-    Y = _sum_partials(lambda q: ops.mlp_tp_fc2_forward_peer(H, lo, B_i, T, h, fs, q, ws), b, T, h, dev,
-                      group=group, sequence_parallel=sequence_parallel, reduction=reduction, exchange=exchange,
-                      ws=ws, ops=ops)
+    if mode == binding.FP8:
+        # fp16 H with its e4m3 residual; the fp16 copy of B_i lives in the workspace
+        ws = ops.make_workspace_mode(T, h, fs, 1, binding.FP8, device=dev)
+        f16, e4m3 = _fp8_dtypes(ops)
+        H = torch.empty(T, fs, dtype=f16, device=dev)
+        H_lo = torch.empty(T, fs, dtype=e4m3, device=dev)
+        ops.mlp_tp_fp8_prepare_forward(B_i, T, h, fs, 1, ws)
+        ops.mlp_tp_fc1_forward_fp8(X, A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws)
+        gemm = lambda q: ops.mlp_tp_fc2_forward_peer_fp8(H, T, h, fs, q, ws)  # noqa: E731
+    else:
+        ws = ops.make_workspace(T, h, fs, 1, dev)
+        H = torch.empty(T, fs, dtype=dt, device=dev)
+        H_lo = torch.empty(T, fs, dtype=dt, device=dev)
+        ops.mlp_tp_fc1_forward(X, A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws)
+        lo = None if mode & binding.FAST_FC2_FORWARD else H_lo
+        gemm = lambda q: ops.mlp_tp_fc2_forward_peer(H, lo, B_i, T, h, fs, q, ws)  # noqa: E731
+    Y = _sum_partials(gemm, b, T, h, dev, group=group, sequence_parallel=sequence_parallel, reduction=reduction,
+                      exchange=exchange, ws=ws, ops=ops)
     return Y, Saved(X, Z, H, H_lo, ws, exchange, owns)
 
 
@@ -221,19 +242,33 @@ def backward(dY: torch.Tensor, saved: Saved, A_i: torch.Tensor, B_i: torch.Tenso
     dt, _ = _dtypes(ops)
     dev = dY.device
     e = lambda *s: torch.empty(*s, dtype=dt, device=dev)  # noqa: E731
-    dH, dH_lo, da = e(T, fs), e(T, fs), e(fs)
-    ops.mlp_tp_fc2_backward_data(dY, B_i, saved.Z, T, h, fs, 1, dH, dH_lo, da, saved.ws)
-    dB, db = e(fs, h), e(h)
-    ops.mlp_tp_fc2_backward_weight(saved.H, saved.H_lo, dY, T, h, fs, 1, dB, db, saved.ws)
-    lo = None if mode & binding.FAST_FC1_BACKWARD_DATA else dH_lo
+    da, dB, db = e(fs), e(fs, h), e(h)
+    fp8 = mode == binding.FP8
+    if fp8:
+        # statistics, scales and the fp16 / e4m3 copies of X, dY and A_i in the workspace
+        f16, e4m3 = _fp8_dtypes(ops)
+        dH = torch.empty(T, fs, dtype=f16, device=dev)
+        dH_lo = torch.empty(T, fs, dtype=e4m3, device=dev)
+        ops.mlp_tp_fp8_prepare_backward(dY, saved.X, A_i, B_i, T, h, fs, 1, saved.ws)
+        ops.mlp_tp_fc2_backward_data_fp8(dY, B_i, saved.Z, T, h, fs, 1, dH, dH_lo, da, saved.ws)
+        ops.mlp_tp_fc2_backward_weight_fp8(saved.H, saved.H_lo, dY, T, h, fs, 1, dB, db, saved.ws)
+        gemm = lambda q: ops.mlp_tp_fc1_backward_data_peer_fp8(dH, T, h, fs, q, saved.ws)  # noqa: E731
+    else:
+        dH, dH_lo = e(T, fs), e(T, fs)
+        ops.mlp_tp_fc2_backward_data(dY, B_i, saved.Z, T, h, fs, 1, dH, dH_lo, da, saved.ws)
+        ops.mlp_tp_fc2_backward_weight(saved.H, saved.H_lo, dY, T, h, fs, 1, dB, db, saved.ws)
+        lo = None if mode & binding.FAST_FC1_BACKWARD_DATA else dH_lo
+        gemm = lambda q: ops.mlp_tp_fc1_backward_data_peer(dH, lo, A_i, T, h, fs, q, saved.ws)  # noqa: E731
     exchange, owns = saved.exchange, saved.owns_exchange
     if reduction == "peer" and exchange is None:
         exchange, owns = PeerExchange(T, h, group, dev, ops), True
-    dX = _sum_partials(lambda q: ops.mlp_tp_fc1_backward_data_peer(dH, lo, A_i, T, h, fs, q, saved.ws), None,
-                       T, h, dev, group=group, sequence_parallel=sequence_parallel, reduction=reduction,
-                       exchange=exchange, ws=saved.ws, ops=ops)
+    dX = _sum_partials(gemm, None, T, h, dev, group=group, sequence_parallel=sequence_parallel,
+                       reduction=reduction, exchange=exchange, ws=saved.ws, ops=ops)
     dA = e(h, fs)
-    ops.mlp_tp_fc1_backward_weight(saved.X, dH, dH_lo, T, h, fs, 1, dA, saved.ws)
+    if fp8:
+        ops.mlp_tp_fc1_backward_weight_fp8(dH, dH_lo, T, h, fs, 1, dA, saved.ws)
+    else:
+        ops.mlp_tp_fc1_backward_weight(saved.X, dH, dH_lo, T, h, fs, 1, dA, saved.ws)
     if owns:
         # the exchange's buffers are read by this rank's last reduce and by the
         # other ranks' GEMMs: every rank syncs and meets before it unmaps

@@ -56,3 +56,10 @@ def test_bench_line_keeps_the_contract():
     assert isinstance(j["clocks"]["reasons"], list)
     assert j["precision_mode"]["timed"] == "fast" and j["accurate"]["value"] > 0
     assert j["steady"]["seconds"] >= bench.STEADY_SECONDS * 0.9
+    # the fp16 + e4m3 mode's leg: same FLOPs per step, its eight stage calls timed one by one
+    f8 = j["fp8"]
+    assert abs(f8["value"] - wl.flops / (f8["ms_per_step"] * 1e-3) / 1e12) <= 1e-6 * f8["value"]
+    assert set(f8["stage_ms"]) == set(bench.FP8_STAGES) and f8["tensor_units_per_step"] == 7
+    d = f8["dominant"]
+    assert d["stage"] in bench.FP8_STAGE_PRODUCTS and abs(d["frac"] - d["achieved"] / d["peak"]) < 1e-9
+    assert f8["gpu_launches"] > 0 and f8["gpu_launches"] % steps == 0

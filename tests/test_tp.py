@@ -82,7 +82,7 @@ def _run(world, shape, sp, mode):
 
 
 @pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
-@pytest.mark.parametrize("mode", [0, 3], ids=["accurate", "fast"])
+@pytest.mark.parametrize("mode", [0, 3, 4], ids=["accurate", "fast", "fp8"])
 def test_two_ranks_match_the_unsharded_block(sp, mode):
     res = _run(2, (64, 128, 256), sp, mode)
     assert set(res) == {0, 1}

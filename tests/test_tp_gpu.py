@@ -53,7 +53,7 @@ def _worker(port, sp, mode, reduction, results):
 
 
 @pytest.mark.parametrize("sp", [False, True], ids=["tensor_parallel", "sequence_parallel"])
-@pytest.mark.parametrize("mode", [0, 3], ids=["accurate", "fast"])
+@pytest.mark.parametrize("mode", [0, 3, 4], ids=["accurate", "fast", "fp8"])
 @pytest.mark.parametrize("reduction", ["peer", "nccl"])
 def test_one_rank_through_the_library_meets_the_bar(sp, mode, reduction):
     ctx = mp.get_context("spawn")

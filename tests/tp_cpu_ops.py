@@ -93,3 +93,45 @@ def mlp_tp_fc1_backward_data_peer(dH, dH_lo, A, T, h, fs, peer, ws, stream=None)
 def mlp_tp_peer_reduce(peer, bias, T, h, out, ws, stream=None):
     s = _np(peer.recv[0])[:T]
     out.copy_(torch.from_numpy(s + (_np(bias) if bias is not None else 0.0)))
+
+
+# ---- the fp16 + e4m3 mode's calls (the library keeps dH scaled by a power of
+# two between its stages; this stand-in keeps the scale 1, all in fp64)
+F16_DTYPE = torch.float64
+E4M3_DTYPE = torch.float64
+
+
+def make_workspace_mode(T, h, f, t, mode, recompute=False, device=None):
+    return {}  # the prepare calls leave the weight and input copies here
+
+
+def mlp_tp_fp8_prepare_forward(B, T, h, f, t, ws, stream=None):
+    ws["B"] = B
+
+
+def mlp_tp_fp8_prepare_backward(dY, X, A, B, T, h, f, t, ws, stream=None):
+    ws["A"], ws["X"] = A, X
+
+
+def mlp_tp_fc1_forward_fp8(X, A, a, T, h, f, t, Z, H, H_lo, ws, stream=None):
+    mlp_tp_fc1_forward(X, A, a, T, h, f, t, Z, H, H_lo, ws)
+
+
+def mlp_tp_fc2_forward_peer_fp8(H, T, h, fs, peer, ws, stream=None):
+    peer.recv[0].copy_(torch.from_numpy(_np(H) @ _np(ws["B"])))
+
+
+def mlp_tp_fc2_backward_data_fp8(dY, B, Z, T, h, f, t, dH, dH_lo, da, ws, stream=None):
+    mlp_tp_fc2_backward_data(dY, B, Z, T, h, f, t, dH, dH_lo, da, ws)
+
+
+def mlp_tp_fc2_backward_weight_fp8(H, H_lo, dY, T, h, f, t, dB, db, ws, stream=None):
+    mlp_tp_fc2_backward_weight(H, H_lo, dY, T, h, f, t, dB, db, ws)
+
+
+def mlp_tp_fc1_backward_data_peer_fp8(dH, T, h, fs, peer, ws, stream=None):
+    peer.recv[0].copy_(torch.from_numpy(_np(dH) @ _np(ws["A"]).T))
+
+
+def mlp_tp_fc1_backward_weight_fp8(dH, dH_lo, T, h, f, t, dA, ws, stream=None):
+    mlp_tp_fc1_backward_weight(ws["X"], dH, dH_lo, T, h, f, t, dA, ws)
