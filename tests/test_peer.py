@@ -122,6 +122,58 @@ def test_emulated_ranks_sum_to_the_unsharded_block(N, mode):
             assert np.all(counters == epoch * N * 8) and np.all(consumed == epoch), o
 
 
+def _activations_fp8(inp, A_i, a_i, B_i, T, h, fs):
+    """This rank's fp16 + e4m3 activations; the forward's workspace keeps the
+    fp16 copy of B_i, the backward's the copy of A_i and the statistics."""
+    FP8 = binding.FP8
+    ws_f, ws_b = (binding.make_workspace_mode(T, h, fs, 1, FP8) for _ in range(2))
+    Z = torch.empty(T, fs, dtype=torch.float32, device="cuda")
+    H, dH = (torch.empty(T, fs, dtype=torch.float16, device="cuda") for _ in range(2))
+    H_lo, dH_lo = (torch.empty(T, fs, dtype=torch.uint8, device="cuda") for _ in range(2))
+    binding.mlp_tp_fp8_prepare_forward(B_i, T, h, fs, 1, ws_f)
+    binding.mlp_tp_fc1_forward_fp8(inp["X"], A_i, a_i, T, h, fs, 1, Z, H, H_lo, ws_f)
+    binding.mlp_tp_fp8_prepare_backward(inp["dY"], inp["X"], A_i, B_i, T, h, fs, 1, ws_b)
+    binding.mlp_tp_fc2_backward_data_fp8(inp["dY"], B_i, Z, T, h, fs, 1, dH, dH_lo, None, ws_b)
+    binding.mlp_tp_check(ws_f)
+    binding.mlp_tp_check(ws_b)
+    return {"H": H, "dH": dH, "ws_f": ws_f, "ws_b": ws_b}
+
+
+def test_emulated_ranks_fp8_mode():
+    """Four ranks in the fp16 + e4m3 mode: each rank's sH follows from its own
+    shard of B, the partials leave the epilogue unscaled, and the owners' sums
+    meet the bar against the unsharded block."""
+    N = 4
+    T, h, f = 1024, 384, 2048
+    fs = f // N
+    rb, fb = binding.peer_recv_bytes(T, h, N), binding.peer_flag_bytes(T, h, N)
+    recv = [_zeros_bytes(rb) for _ in range(N)]
+    flags = [_zeros_bytes(fb) for _ in range(N)]
+    rows = T // N
+    host = inputs.make_custom(T, h, f, seed=31)
+    inp = {k: v.cuda() for k, v in host.items()}
+    ref = oracle.full(host)
+    shards = [tp.shard_parameters(inp["A"], inp["a"], inp["B"], r, N) for r in range(N)]
+    acts = [_activations_fp8(inp, A_i, a_i, B_i, T, h, fs) for (A_i, a_i, B_i) in shards]
+    for epoch, what in ((1, "Y"), (2, "dX")):
+        qs = [binding.make_peer(r, N, recv, flags, epoch) for r in range(N)]
+        for r in range(N):
+            a = acts[r]
+            if what == "Y":
+                binding.mlp_tp_fc2_forward_peer_fp8(a["H"], T, h, fs, qs[r], a["ws_f"])
+            else:
+                binding.mlp_tp_fc1_backward_data_peer_fp8(a["dH"], T, h, fs, qs[r], a["ws_b"])
+        outs = []
+        for o in range(N):
+            out = torch.empty(rows, h, dtype=torch.bfloat16, device="cuda")
+            binding.mlp_tp_peer_reduce(qs[o], inp["b"] if what == "Y" else None, T, h, out, acts[o]["ws_f"])
+            outs.append(out)
+        for a in acts:
+            binding.mlp_tp_check(a["ws_f"])
+            binding.mlp_tp_check(a["ws_b"])
+        assert_close(f"{what} over {N} ranks (fp8 mode)", torch.cat(outs, dim=0), ref[what])
+
+
 def test_bounded_waits_report_timeout_and_the_context_survives():
     T, h, f = 256, 256, 512
     inp = {k: v.cuda() for k, v in inputs.make_custom(T, h, f, seed=9).items()}
