@@ -34,6 +34,11 @@ peak is the measured burst bf16 figure unless the SM clock sampled while the
 stages were timed sat clearly below its maximum (median < 0.97·max), when it
 is the measured sustained figure.
 
+`fp8` times the fp16 + e4m3 mode (MLP_TP_FP8: fp16 operands, e4m3 residual
+products in the weight gradients) through its stage calls, with its own
+per-stage times and dominant-stage roofline; the headline stays on the bf16
+modes.
+
 `steady` times the same step loop for at least two seconds, long enough for
 the clock to settle under the power cap; both it and the headline report the
 median SM clock and ms-per-step × MHz.
@@ -567,7 +572,8 @@ def main():
                "tensor_units_per_step": sum(FP8_STAGE_PRODUCTS.values()),
                "dominant": {"stage": dom, "achieved": ach, "peak": pk, "frac": ach / pk,
                             "peak_source": src8 + (" bf16_tflops_sustained" if settled else " bf16_tflops (burst)"),
-                            "executed_tflops": ach * FP8_STAGE_PRODUCTS[dom], "stage_clocks": ck},
+                            "executed_tflops": ach * FP8_STAGE_PRODUCTS[dom], "stage_clocks": ck,
+                            "traffic": traffic_for("fp8." + dom, wl, t) if args.tokens is None else None},
                "api": "mlp_tp_fp8_prepare_forward, the two forward stages, mlp_tp_fp8_prepare_backward and the "
                       "four backward stages of MLP_TP_FP8 (fp16 operands, e4m3 residual products in dA, dB)"}
 
@@ -925,7 +931,7 @@ def kernel_source_digest():
     roofline reports)."""
     import hashlib
     hsh = hashlib.sha256()
-    for n in ("gemm.cuh", "ptx.cuh", "peer.cuh", "mlp_tp.cu"):
+    for n in ("gemm.cuh", "ptx.cuh", "peer.cuh", "fp8.cuh", "mlp_tp.cu"):
         with open(os.path.join(ROOT, "tensor_transformer_mlp_bias_b200", "csrc", n), "rb") as fh:
             hsh.update(fh.read())
     return hsh.hexdigest()[:12]
