@@ -22,10 +22,13 @@ during the timed region and the number of library kernel launches in it.
 
 Precision mode.  The library's default (accurate) mode takes Y and dX over
 both halves of the bf16 activation pair; the fast mode takes them from the
-high half only.  `--mode auto` times the fast mode on the workloads where its
-GPU parity test meets the bar (tiny, GPT-2-medium, h4096, 175B-class) and the
-accurate mode otherwise; the line says which (`precision_mode`), and with the
-fast mode it also times the accurate mode over as many steps (`accurate`).
+high half only; the fp8 mode (MLP_TP_FP8) keeps H and dH as fp16 plus an
+e4m3 residual, runs dA and dB as an fp16 product plus an e4m3 residual
+product and Y, dX as one fp16 product each.  `--mode auto` times the fastest
+mode whose GPU parity test meets the bar on the workload: the fp8 mode on all
+five.  The line says which (`precision_mode`, `dtype`) and times the bf16
+modes beside it over as many steps (`accurate`; `fast` where its parity test
+passes).
 
 Roofline.  `roofline.achieved` is the dominant stage's algorithmic FLOPs
 (2·T·h·f per GEMM) over its CUDA-event time; `executed_tflops` counts every
@@ -79,15 +82,20 @@ STAGE_KERNEL = {
 # tensor-core products each stage's GEMM runs in the fast mode, in units of 2·T·h·f
 STAGE_PRODUCTS = {"fc1_forward": 1, "fc2_forward": 1, "fc2_backward_data": 1, "fc2_backward_weight": 2,
                   "fc1_backward_data": 1, "fc1_backward_weight": 2}
-MODES = {"accurate": 0, "fast": 3}
+MODES = {"accurate": 0, "fast": 3, "fp8": 4}
 # workloads whose GPU parity test runs the fast mode and meets the bar
 FAST_MODE_PARITY = ("tiny", "gpt2-medium", "h4096", "175b-class")
+# workloads whose GPU parity test runs the fp16 + e4m3 mode and meets the bar (tests/test_fp8.py)
+FP8_MODE_PARITY = ("tiny", "gpt2-medium", "h4096", "8.3b-class", "175b-class")
 STEADY_SECONDS = 2.0
 
 
 def stage_products(mode):
     """Tensor-core products per stage for a precision mode (flags 1 and 2
-    drop the low half from the Y and dX GEMMs)."""
+    drop the low half from the Y and dX GEMMs; the fp8 mode's weight
+    gradients take 1.5 bf16-products of tensor time)."""
+    if mode == MODES["fp8"]:
+        return dict(FP8_STAGE_PRODUCTS)
     p = dict(STAGE_PRODUCTS)
     p["fc2_forward"] += 0 if mode & 1 else 1
     p["fc1_backward_data"] += 0 if mode & 2 else 1
@@ -95,9 +103,52 @@ def stage_products(mode):
 
 
 def pick_mode(arg, wl_name):
+    """auto: the fastest mode whose GPU parity test meets the bar on this workload."""
     if arg == "auto":
+        if wl_name in FP8_MODE_PARITY:
+            return "fp8"
         return "fast" if wl_name in FAST_MODE_PARITY else "accurate"
     return arg
+
+
+def make_buffers(torch, T, h, f):
+    """Outputs and activations of one step, for every precision mode."""
+    e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device="cuda")  # noqa: E731
+    return {"Z": e(T, f, dt=torch.float32), "H": e(T, f), "H_lo": e(T, f), "dH": e(T, f), "dH_lo": e(T, f),
+            "H16": e(T, f, dt=torch.float16), "H8": e(T, f, dt=torch.uint8), "dH16": e(T, f, dt=torch.float16),
+            "dH8": e(T, f, dt=torch.uint8), "Y": e(T, h), "dX": e(T, h), "dA": e(h, f), "dB": e(f, h), "da": e(f),
+            "db": e(h)}
+
+
+def stage_calls(binding, mode_name, dev, b, T, h, f, t, ws, sh):
+    """(stage names, calls) of one step in a precision mode; `sh` None runs
+    them on the current stream (graph capture)."""
+    if mode_name == "fp8":
+        return FP8_STAGES, (
+            lambda: binding.mlp_tp_fp8_prepare_forward(dev["B"], T, h, f, t, ws, sh),
+            lambda: binding.mlp_tp_fc1_forward_fp8(dev["X"], dev["A"], dev["a"], T, h, f, t, b["Z"], b["H16"],
+                                                   b["H8"], ws, sh),
+            lambda: binding.mlp_tp_fc2_forward_fp8(b["H16"], dev["b"], T, h, f, t, b["Y"], ws, sh),
+            lambda: binding.mlp_tp_fp8_prepare_backward(dev["dY"], dev["X"], dev["A"], dev["B"], T, h, f, t, ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_data_fp8(dev["dY"], dev["B"], b["Z"], T, h, f, t, b["dH16"], b["dH8"],
+                                                         b["da"], ws, sh),
+            lambda: binding.mlp_tp_fc2_backward_weight_fp8(b["H16"], b["H8"], dev["dY"], T, h, f, t, b["dB"], b["db"],
+                                                           ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_data_fp8(b["dH16"], T, h, f, t, b["dX"], ws, sh),
+            lambda: binding.mlp_tp_fc1_backward_weight_fp8(b["dH16"], b["dH8"], T, h, f, t, b["dA"], ws, sh),
+        )
+    mode = MODES[mode_name]
+    lo_y = None if mode & 1 else b["H_lo"]
+    lo_dx = None if mode & 2 else b["dH_lo"]
+    return STAGES, (
+        lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, b["Z"], b["H"], b["H_lo"], ws, sh),
+        lambda: binding.mlp_tp_fc2_forward(b["H"], lo_y, dev["B"], dev["b"], T, h, f, t, b["Y"], ws, sh),
+        lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], b["Z"], T, h, f, t, b["dH"], b["dH_lo"], b["da"],
+                                                 ws, sh),
+        lambda: binding.mlp_tp_fc2_backward_weight(b["H"], b["H_lo"], dev["dY"], T, h, f, t, b["dB"], b["db"], ws, sh),
+        lambda: binding.mlp_tp_fc1_backward_data(b["dH"], lo_dx, dev["A"], T, h, f, t, b["dX"], ws, sh),
+        lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], b["dH"], b["dH_lo"], T, h, f, t, b["dA"], ws, sh),
+    )
 
 
 def roofline_entry(stage_ms, mode, T, h, f, clocks, peaks, peak_src):
@@ -107,7 +158,7 @@ def roofline_entry(stage_ms, mode, T, h, f, clocks, peaks, peak_src):
     unless the SM clock sampled while the stages were timed sat below 0.97 of
     its maximum, then the measured sustained one."""
     products = stage_products(mode)
-    dom = max(STAGES, key=lambda k: stage_ms[k])
+    dom = max((k for k in stage_ms if k in products), key=lambda k: stage_ms[k])  # GEMM stages only
     unit = 2.0 * T * h * f
     secs = stage_ms[dom] * 1e-3
     achieved = unit / secs / 1e12
@@ -119,7 +170,8 @@ def roofline_entry(stage_ms, mode, T, h, f, clocks, peaks, peak_src):
     kind = ("bf16_tflops_sustained (SM clock median %.0f of %.0f MHz while the stages were timed)" % (mhz, mx)
             if settled else "bf16_tflops (burst; SM clock median %s of %s MHz while the stages were timed)"
             % (mhz, mx))
-    return {"bound": "tensor", "kernel": STAGE_KERNEL[dom], "stage": dom, "achieved": achieved, "peak": peak,
+    kernels = FP8_STAGE_KERNEL if mode == MODES["fp8"] else STAGE_KERNEL
+    return {"bound": "tensor", "kernel": kernels[dom], "stage": dom, "achieved": achieved, "peak": peak,
             "unit": UNIT, "frac": achieved / peak, "peak_source": f"{peak_src} {kind}",
             "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
             "algorithmic_flops_per_launch": unit, "avg_launch_ms": stage_ms[dom],
@@ -135,6 +187,14 @@ FP8_STAGES = ("fp8_prepare_forward", "fc1_forward", "fc2_forward", "fp8_prepare_
 # bf16 product of K = 16)
 FP8_STAGE_PRODUCTS = {"fc1_forward": 1, "fc2_forward": 1, "fc2_backward_data": 1, "fc2_backward_weight": 1.5,
                       "fc1_backward_data": 1, "fc1_backward_weight": 1.5}
+FP8_STAGE_KERNEL = {
+    "fc1_forward": "Z=X·A+a, H=GeLU(Z) as fp16 + e4m3 residual (column-parallel GEMM, bias+GeLU epilogue)",
+    "fc2_forward": "Y=Σ_i H16_i·B16_i + b (row-parallel GEMM, fp16 operands, shard-sum epilogue)",
+    "fc2_backward_data": "dH=(dY·Bᵀ)⊙GeLU'(Z) as scaled fp16 + e4m3 residual, da (GEMM) + da reduce",
+    "fc2_backward_weight": "dB=(H16ᵀ·dY16 + H8ᵀ·dY8)/sY (fp16 product + e4m3 residual product) + db column sum",
+    "fc1_backward_data": "dX=Σ_i dH16_i·A16_iᵀ/sH (GEMM, fp16 operands, shard-sum epilogue)",
+    "fc1_backward_weight": "dA=(X16ᵀ·dH16 + X8ᵀ·dH8)/(sX·sH) (fp16 product + e4m3 residual product)",
+}
 
 
 def fp8_leg(binding, dev, T, h, f, t, steps, stream, clock_interval_ms, local, check_every=None):
@@ -407,9 +467,10 @@ def main():
                     help="override the workload's token count (small profiling captures of the large workloads; "
                          "the headline uses the workload's own T)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--mode", default="auto", choices=["auto", "fast", "accurate"],
+    ap.add_argument("--mode", default="auto", choices=["auto", "fp8", "fast", "accurate"],
                     help="precision mode: accurate (library default: Y and dX over the bf16 pair), fast (Y and dX "
-                         "from the high half), auto (fast where its parity test meets the bar, else accurate)")
+                         "from the high half), fp8 (fp16 operands with e4m3 residual products), auto (the fastest "
+                         "mode whose parity test meets the bar on the workload)")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of each end-to-end leg (default: --steps, so it runs as long as the headline loop)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -422,7 +483,7 @@ def main():
                     help="steps of the per-stage timing pass (default: enough for 0.3 s; small for ncu captures)")
     ap.add_argument("--no-fp8-leg", action="store_true", help="skip timing the fp16 + e4m3 mode")
     ap.add_argument("--no-accurate-leg", action="store_true",
-                    help="with the fast mode timed, skip timing the accurate mode beside it")
+                    help="skip timing the bf16 modes (accurate, fast) beside the timed one")
     ap.add_argument("--clock-interval-ms", type=int, default=50,
                     help="nvidia-smi sampling period during the timed region")
     args = ap.parse_args()
@@ -456,27 +517,15 @@ def main():
     T, h, f, t = wl.T, wl.h, wl.f, args.t
     host = inputs.make_inputs(wl, seed=wl.seed + rank)
     dev = {k: v.cuda() for k, v in host.items()}
-    e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
-    Z = torch.empty(T, f, dtype=torch.float32, device="cuda")
-    H, H_lo, Y, dH, dH_lo = e(T, f), e(T, f), e(T, h), e(T, f), e(T, f)
-    dX, dA, dB, da, db = e(T, h), e(h, f), e(f, h), e(f), e(h)
+    bufs = make_buffers(torch, T, h, f)
     mode_name = pick_mode(args.mode, wl.name)
     mode = MODES[mode_name]
-    H_lo2 = None if mode & 1 else H_lo
-    dH_lo2 = None if mode & 2 else dH_lo
-    ws = binding.make_workspace(T, h, f, t)
+    ws = binding.make_workspace_mode(T, h, f, t, MODES["fp8"])  # large enough for every mode
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
+    stage_names, head_calls = stage_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, sh)
 
-    def step(evs=None, lo_y=H_lo2, lo_dx=dH_lo2):
-        calls = (
-            lambda: binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, H_lo, ws, sh),
-            lambda: binding.mlp_tp_fc2_forward(H, lo_y, dev["B"], dev["b"], T, h, f, t, Y, ws, sh),
-            lambda: binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, dH_lo, da, ws, sh),
-            lambda: binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t, dB, db, ws, sh),
-            lambda: binding.mlp_tp_fc1_backward_data(dH, lo_dx, dev["A"], T, h, f, t, dX, ws, sh),
-            lambda: binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t, dA, ws, sh),
-        )
+    def step(evs=None, calls=head_calls):
         for i, c in enumerate(calls):
             if evs is not None:
                 evs[i].record(stream)
@@ -512,7 +561,7 @@ def main():
     # per-stage times (events between the stage calls), with the clocks of
     # this window: the roofline's peak follows them
     n_ev = args.stage_steps or max(10, args.steps // 4, int(0.3e3 / max(local_ms / args.steps, 1e-3)) + 1)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(n_ev)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)] for _ in range(n_ev)]
     torch.cuda.synchronize()
     with ClockSampler(local, args.clock_interval_ms) as clk_stages:
         for k in range(n_ev):
@@ -520,7 +569,7 @@ def main():
         torch.cuda.synchronize()
     binding.mlp_tp_check(ws, sh)
     stage_ms = {s: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(n_ev))
-                for i, s in enumerate(STAGES)}
+                for i, s in enumerate(stage_names)}
     max_ms, total_flops = reduce_max_sum(local_ms, float(wl.flops) * args.steps)
     value = total_flops / (max_ms * 1e-3) / 1e12
     ms_per_step = max_ms / args.steps
@@ -542,20 +591,26 @@ def main():
         ms_l, fl_l = reduce_max_sum(s_l.elapsed_time(e_l), float(wl.flops) * n)
         return ms_l, fl_l, c.summary()
 
-    # ------------------------------------------------ the accurate (default) mode beside the fast one
-    accurate = None
-    if mode != MODES["accurate"] and not args.no_accurate_leg:
+    # ------------------------------------------------ the bf16 modes beside the timed one
+    # accurate (the library's default) always; fast where its parity test meets the bar
+    other_modes = {}
+    for leg in ("accurate", "fast"):
+        if leg == mode_name or args.no_accurate_leg or (leg == "fast" and wl.name not in FAST_MODE_PARITY):
+            continue
+        _, leg_calls = stage_calls(binding, leg, dev, bufs, T, h, f, t, ws, sh)
         for _ in range(3):
-            step(lo_y=H_lo, lo_dx=dH_lo)
-        ms_a, fl_a, clk_a = timed_loop(args.steps, lo_y=H_lo, lo_dx=dH_lo)
-        accurate = {"value": fl_a / (ms_a * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_a / args.steps,
-                    "steps": args.steps, "clocks": clk_a,
-                    "api": "the same stage calls with the low half of the pair in the Y and dX GEMMs "
-                           "(the library's default mode)"}
+            step(calls=leg_calls)
+        ms_a, fl_a, clk_a = timed_loop(args.steps, calls=leg_calls)
+        other_modes[leg] = {
+            "value": fl_a / (ms_a * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_a / args.steps,
+            "steps": args.steps, "clocks": clk_a,
+            "api": ("the six bf16 stage calls with the low half of the pair in the Y and dX GEMMs (the library's "
+                    "default mode)" if leg == "accurate" else
+                    "the six bf16 stage calls with Y and dX from the high half of the pair (fast mode)")}
 
-    # ------------------------------------------------ the fp16 + e4m3 mode (MLP_TP_FP8) beside them
+    # ------------------------------------------------ the fp16 + e4m3 mode (MLP_TP_FP8) beside a bf16 headline
     fp8 = None
-    if not args.no_fp8_leg and world == 1:
+    if not args.no_fp8_leg and world == 1 and mode_name != "fp8":
         r8 = fp8_leg(binding, dev, T, h, f, t, args.steps, stream, args.clock_interval_ms, local)
         peaks8, src8 = load_peaks()
         gemm_stages = [k for k in r8["stage_ms"] if k in FP8_STAGE_PRODUCTS]
@@ -616,14 +671,20 @@ def main():
         peer_hbm = None
         recv = torch.zeros(binding.peer_recv_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
         flags = torch.zeros(binding.peer_flag_bytes(T, h, 1), dtype=torch.uint8, device="cuda")
-        ws_p = binding.make_workspace(T, h, f, 1)
+        ws_p = binding.make_workspace_mode(T, h, f, 1, MODES["fp8"])
         Yp = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+        if mode_name == "fp8":
+            binding.mlp_tp_fp8_prepare_forward(dev["B"], T, h, f, 1, ws_p, sh)
+            peer_gemm = lambda q: binding.mlp_tp_fc2_forward_peer_fp8(bufs["H16"], T, h, f, q, ws_p, sh)  # noqa: E731
+        else:
+            lo_p = None if mode & 1 else bufs["H_lo"]
+            peer_gemm = lambda q: binding.mlp_tp_fc2_forward_peer(bufs["H"], lo_p, dev["B"], T, h, f, q, ws_p, sh)  # noqa: E731
         n_p = max(10, args.steps)
         evp = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_p + 3)]
         for k in range(n_p + 3):
             q = binding.make_peer(0, 1, [recv], [flags], k + 1)
             evp[k][0].record(stream)
-            binding.mlp_tp_fc2_forward_peer(H, H_lo2, dev["B"], T, h, f, q, ws_p, sh)
+            peer_gemm(q)
             evp[k][1].record(stream)
             binding.mlp_tp_peer_reduce(q, dev["b"], T, h, Yp, ws_p, sh)
             evp[k][2].record(stream)
@@ -634,11 +695,12 @@ def main():
         rbytes = 4.0 * T * h + 2.0 * T * h + 2.0 * h
         peaks_p, _ = load_peaks()
         peer_hbm = float(peaks_p.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        peer = {"gemm_ms": g_ms, "gemm_tflops": 2.0 * T * h * f * (1 if mode & 1 else 2) / (g_ms * 1e-3) / 1e12,
+        peer = {"gemm_ms": g_ms, "gemm_tflops": 2.0 * T * h * f * stage_products(mode)["fc2_forward"] / (g_ms * 1e-3) / 1e12,
                 "reduce_ms": r_ms, "reduce_gbs": rbytes / (r_ms * 1e-3) / 1e9,
                 "reduce_frac_of_hbm": rbytes / (r_ms * 1e-3) / 1e9 / peer_hbm, "hbm_peak_gbs": peer_hbm,
                 "reduce_bytes": rbytes, "steps": n_p,
-                "api": "mlp_tp_fc2_forward_peer + mlp_tp_peer_reduce, one rank (world = 1), flags on; "
+                "api": ("mlp_tp_fc2_forward_peer_fp8" if mode_name == "fp8" else "mlp_tp_fc2_forward_peer")
+                       + " + mlp_tp_peer_reduce, one rank (world = 1), flags on; "
                        "gemm_tflops counts the tensor products the GEMM runs"}
         del recv, flags, ws_p
 
@@ -649,15 +711,12 @@ def main():
     for t_other in wl.shards:
         if t_other == t or args.no_per_t:
             continue
-        ws_o = binding.make_workspace(T, h, f, t_other)
+        ws_o = binding.make_workspace_mode(T, h, f, t_other, MODES["fp8"])
+        _, calls_o = stage_calls(binding, mode_name, dev, bufs, T, h, f, t_other, ws_o, sh)
 
         def step_o():
-            binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t_other, Z, H, H_lo, ws_o, sh)
-            binding.mlp_tp_fc2_forward(H, H_lo2, dev["B"], dev["b"], T, h, f, t_other, Y, ws_o, sh)
-            binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t_other, dH, dH_lo, da, ws_o, sh)
-            binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t_other, dB, db, ws_o, sh)
-            binding.mlp_tp_fc1_backward_data(dH, dH_lo2, dev["A"], T, h, f, t_other, dX, ws_o, sh)
-            binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t_other, dA, ws_o, sh)
+            for c in calls_o:
+                c()
 
         for _ in range(3):
             step_o()
@@ -682,13 +741,11 @@ def main():
     # maps, launch calls), which is what bounds the smallest batches.
     graph = None
     if not args.no_graph:
+        _, calls_g = stage_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, None)
+
         def step_current_stream():
-            binding.mlp_tp_fc1_forward(dev["X"], dev["A"], dev["a"], T, h, f, t, Z, H, H_lo, ws)
-            binding.mlp_tp_fc2_forward(H, H_lo2, dev["B"], dev["b"], T, h, f, t, Y, ws)
-            binding.mlp_tp_fc2_backward_data(dev["dY"], dev["B"], Z, T, h, f, t, dH, dH_lo, da, ws)
-            binding.mlp_tp_fc2_backward_weight(H, H_lo, dev["dY"], T, h, f, t, dB, db, ws)
-            binding.mlp_tp_fc1_backward_data(dH, dH_lo2, dev["A"], T, h, f, t, dX, ws)
-            binding.mlp_tp_fc1_backward_weight(dev["X"], dH, dH_lo, T, h, f, t, dA, ws)
+            for c in calls_g:
+                c()
 
         side = torch.cuda.Stream()
         side.wait_stream(stream)
@@ -714,7 +771,7 @@ def main():
         binding.mlp_tp_check(ws, sh)
         ms_g, fl_g = reduce_max_sum(s_g.elapsed_time(e_g), float(wl.flops) * n_g)
         graph = {"value": fl_g / (ms_g * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_g / n_g, "steps": n_g,
-                 "api": "the six stage calls of one step captured once in a CUDA graph and replayed"}
+                 "api": "the stage calls of one step captured once in a CUDA graph and replayed"}
         del cg
 
     # ------------------------------------------------ activation recomputation
@@ -724,13 +781,13 @@ def main():
     # only (the rerun GEMM is overhead, not work).
     recompute = None
     if not args.no_recompute:
-        ws_r = binding.make_recompute_workspace(T, h, f, t)
+        ws_r = binding.make_workspace_mode(T, h, f, t, mode, recompute=True)
 
         def step_r():
             binding.mlp_tp_forward_recompute(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, mode,
-                                             Y, ws_r, sh)
+                                             bufs["Y"], ws_r, sh)
             binding.mlp_tp_backward_recompute(dev["dY"], dev["X"], dev["A"], dev["a"], dev["B"], T, h, f, t, mode,
-                                              dX, dA, da, dB, db, ws_r, sh)
+                                              bufs["dX"], bufs["dA"], bufs["da"], bufs["dB"], bufs["db"], ws_r, sh)
 
         for _ in range(3):
             step_r()
@@ -759,6 +816,7 @@ def main():
     # step k+1 and the device->host copy of step k-1 overlap the compute of
     # step k.  The timed region spans the first copy in to the last copy out.
     pin = {k: v.pin_memory() for k, v in host.items()}
+    H_e, Hlo_e = (bufs["H16"], bufs["H8"]) if mode_name == "fp8" else (bufs["H"], bufs["H_lo"])
     out_names = ("Y", "dX", "dA", "da", "dB", "db")
     out_shapes = {"Y": (T, h), "dX": (T, h), "dA": (h, f), "da": (f,), "dB": (f, h), "db": (h,)}
     sets = []
@@ -791,8 +849,8 @@ def main():
                 s_cmp.wait_event(out_done[k - 2])  # step k-2's outputs in set k % 2 copied out
             cs = s_cmp.cuda_stream
             binding.mlp_tp_forward(d_in["X"], d_in["A"], d_in["a"], d_in["B"], d_in["b"], T, h, f, t, mode,
-                                   d_out["Y"], Z, H, H_lo, ws, cs)
-            binding.mlp_tp_backward(d_in["dY"], d_in["X"], d_in["A"], d_in["B"], Z, H, H_lo, T, h, f, t, mode,
+                                   d_out["Y"], bufs["Z"], H_e, Hlo_e, ws, cs)
+            binding.mlp_tp_backward(d_in["dY"], d_in["X"], d_in["A"], d_in["B"], bufs["Z"], H_e, Hlo_e, T, h, f, t, mode,
                                     d_out["dX"], d_out["dA"], d_out["da"], d_out["dB"], d_out["db"], ws, cs)
             c_done.record(s_cmp)
             cmp_done.append(c_done)
@@ -851,7 +909,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, bf16)",
+        "vs_baseline": None, "dtype": "bf16+fp16+e4m3" if mode == MODES["fp8"] else "bf16", "data": "synthetic (seeded Gaussian, bf16)",
         "config": dict(workload_config(wl, t, world), precision=precision_note(mode),
                        tensor_flops_per_step=2.0 * T * h * f * sum(products.values())),
         "precision_mode": precision_mode_note(mode_name, args.mode, wl.name),
@@ -871,8 +929,7 @@ def main():
         "clocks": clocks,
         "ms_x_mhz": ms_per_step * clocks["sm_mhz"] if clocks.get("sm_mhz") else None,
     }
-    if accurate is not None:
-        line["accurate"] = accurate
+    line.update(other_modes)
     if fp8 is not None:
         line["fp8"] = fp8
     if steady is not None:
@@ -890,6 +947,10 @@ def main():
 
 
 def precision_note(mode):
+    if mode == MODES["fp8"]:
+        return ("bf16 inputs and outputs, fp32 accumulation; Z saved fp32; H, dH saved as fp16 + e4m3 residual; "
+                "Y, dX from one fp16 product (fp16 copies of B, A); dA, dB from an fp16 product plus an e4m3 "
+                "residual product (kind::f8f6f4) in one accumulator, power-of-two per-tensor scales; da from fp32 dH")
     y = "bf16 H (high half)" if mode & 1 else "(H, H_lo) pair"
     dx = "bf16 dH (high half)" if mode & 2 else "(dH, dH_lo) pair"
     return (f"bf16 inputs, fp32 accumulation; Z saved fp32; Y from {y}; dX from {dx}; dA, dB from the "
@@ -897,6 +958,12 @@ def precision_note(mode):
 
 
 def precision_mode_note(mode_name, requested, wl_name):
+    auto = " (chosen by --mode auto)" if requested == "auto" else ""
+    if mode_name == "fp8":
+        why = (f"fp8 mode (MLP_TP_FP8): fp16 operands, e4m3 residual products in the weight gradients; its GPU "
+               f"parity test on the {wl_name} workload meets the 1e-2·(|oracle|+1) bar{auto}; the bf16 modes are "
+               f"timed beside it in `accurate` (the library's default) and `fast`")
+        return {"timed": mode_name, "note": why}
     if mode_name == "fast":
         why = (f"fast mode: Y and dX from the high half of the bf16 activation pair; its GPU parity test on "
                f"the {wl_name} workload meets the 1e-2·(|oracle|+1) bar"

@@ -60,7 +60,7 @@ def test_traffic_lookup(monkeypatch):
     rows = [ln.split() for ln in open(path).read().splitlines() if ln.strip() and not ln.startswith("#")]
     assert rows
     for stage, wl_name, t, digest, nbytes in rows:
-        assert stage in bench.STAGES and wl_name in inputs.WORKLOADS and t.startswith("t=")
+        assert stage.replace("fp8.", "", 1) in bench.STAGES and wl_name in inputs.WORKLOADS and t.startswith("t=")
         assert len(digest) == 12 and float(nbytes) > 0
     stage, wl_name, t, digest, nbytes = rows[0]
     wl, tt = inputs.WORKLOADS[wl_name], int(t[2:])
@@ -135,10 +135,33 @@ def test_stage_products_follow_the_mode():
     assert acc["fc2_forward"] == acc["fc1_backward_data"] == 2 and fast["fc2_forward"] == fast["fc1_backward_data"] == 1
 
 
-def test_auto_mode_is_fast_only_where_its_parity_test_passes():
-    assert bench.pick_mode("auto", "h4096") == "fast"
-    assert bench.pick_mode("auto", "8.3b-class") == "accurate"
+def test_auto_mode_picks_the_fastest_mode_whose_parity_test_passes():
+    # the fp16 + e4m3 mode meets the bar on all five workloads (tests/test_fp8.py)
+    for name in ("tiny", "gpt2-medium", "h4096", "8.3b-class", "175b-class"):
+        assert bench.pick_mode("auto", name) == "fp8"
     assert bench.pick_mode("accurate", "h4096") == "accurate"
+    assert bench.pick_mode("fast", "h4096") == "fast"
+    # without it, fast only where the fast mode's parity test passes
+    saved = bench.FP8_MODE_PARITY
+    try:
+        bench.FP8_MODE_PARITY = ()
+        assert bench.pick_mode("auto", "h4096") == "fast"
+        assert bench.pick_mode("auto", "8.3b-class") == "accurate"
+    finally:
+        bench.FP8_MODE_PARITY = saved
+
+
+def test_fp8_mode_products_and_roofline():
+    p = bench.stage_products(bench.MODES["fp8"])
+    assert sum(p.values()) == 7 and p["fc1_backward_weight"] == 1.5
+    ms = {s: 0.4 for s in bench.FP8_STAGES}
+    ms["fp8_prepare_backward"] = 9.0   # an HBM-bound preparation stage is never the tensor roofline's kernel
+    ms["fc1_backward_weight"] = 0.526
+    r = bench.roofline_entry(ms, bench.MODES["fp8"], 4096, 4096, 16384, {"sm_mhz": 1965, "sm_max_mhz": 1965},
+                             PEAKS, "measured")
+    assert r["stage"] == "fc1_backward_weight" and r["executed_tensor_products"] == 1.5
+    assert abs(r["achieved"] - 2 * 4096 * 4096 * 16384 / 0.526e-3 / 1e12) < 1e-6
+    assert abs(r["executed_tflops"] - 1.5 * r["achieved"]) < 1e-6 and r["frac"] <= 1.0
 
 
 def test_clock_summary_keeps_only_samples_inside_the_window():
