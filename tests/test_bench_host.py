@@ -137,8 +137,9 @@ def test_stage_products_follow_the_mode():
 
 def test_auto_mode_picks_the_fastest_mode_whose_parity_test_passes():
     # the fp16 + e4m3 mode meets the bar on all five workloads (tests/test_fp8.py)
-    for name in ("tiny", "gpt2-medium", "h4096", "8.3b-class", "175b-class"):
+    for name in ("gpt2-medium", "h4096", "8.3b-class", "175b-class"):
         assert bench.pick_mode("auto", name) == "fp8"
+    assert bench.pick_mode("auto", "tiny") == "fast"  # launch-bound: the fp8 mode's extra launches cost more
     assert bench.pick_mode("accurate", "h4096") == "accurate"
     assert bench.pick_mode("fast", "h4096") == "fast"
     # without it, fast only where the fast mode's parity test passes
