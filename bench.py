@@ -123,6 +123,20 @@ def make_buffers(torch, T, h, f):
             "db": e(h)}
 
 
+def step_calls(binding, mode_name, dev, b, T, h, f, t, ws, sh):
+    """One step through the composite calls a user makes, mlp_tp_forward and
+    mlp_tp_backward, in a precision mode (the fp8 mode runs its operand copies
+    on the library's side stream there)."""
+    mode = MODES[mode_name]
+    H, H_lo = (b["H16"], b["H8"]) if mode_name == "fp8" else (b["H"], b["H_lo"])
+    return (
+        lambda: binding.mlp_tp_forward(dev["X"], dev["A"], dev["a"], dev["B"], dev["b"], T, h, f, t, mode, b["Y"],
+                                       b["Z"], H, H_lo, ws, sh),
+        lambda: binding.mlp_tp_backward(dev["dY"], dev["X"], dev["A"], dev["B"], b["Z"], H, H_lo, T, h, f, t, mode,
+                                        b["dX"], b["dA"], b["da"], b["dB"], b["db"], ws, sh),
+    )
+
+
 def stage_calls(binding, mode_name, dev, b, T, h, f, t, ws, sh):
     """(stage names, calls) of one step in a precision mode; `sh` None runs
     them on the current stream (graph capture)."""
@@ -526,7 +540,9 @@ def main():
     ws = binding.make_workspace_mode(T, h, f, t, MODES["fp8"])  # large enough for every mode
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
-    stage_names, head_calls = stage_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, sh)
+    # timed steps: the composite calls; the per-stage pass: the stage calls
+    stage_names, stage_cs = stage_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, sh)
+    head_calls = step_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, sh)
 
     def step(evs=None, calls=head_calls):
         for i, c in enumerate(calls):
@@ -568,7 +584,7 @@ def main():
     torch.cuda.synchronize()
     with ClockSampler(local, args.clock_interval_ms) as clk_stages:
         for k in range(n_ev):
-            step(ev[k])
+            step(ev[k], calls=stage_cs)
         torch.cuda.synchronize()
     binding.mlp_tp_check(ws, sh)
     stage_ms = {s: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(n_ev))
@@ -600,7 +616,7 @@ def main():
     for leg in ("accurate", "fast"):
         if leg == mode_name or args.no_accurate_leg or (leg == "fast" and wl.name not in FAST_MODE_PARITY):
             continue
-        _, leg_calls = stage_calls(binding, leg, dev, bufs, T, h, f, t, ws, sh)
+        leg_calls = step_calls(binding, leg, dev, bufs, T, h, f, t, ws, sh)
         for _ in range(3):
             step(calls=leg_calls)
         ms_a, fl_a, clk_a = timed_loop(args.steps, calls=leg_calls)
@@ -715,7 +731,7 @@ def main():
         if t_other == t or args.no_per_t:
             continue
         ws_o = binding.make_workspace_mode(T, h, f, t_other, MODES["fp8"])
-        _, calls_o = stage_calls(binding, mode_name, dev, bufs, T, h, f, t_other, ws_o, sh)
+        calls_o = step_calls(binding, mode_name, dev, bufs, T, h, f, t_other, ws_o, sh)
 
         def step_o():
             for c in calls_o:
@@ -744,7 +760,7 @@ def main():
     # maps, launch calls), which is what bounds the smallest batches.
     graph = None
     if not args.no_graph:
-        _, calls_g = stage_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, None)
+        calls_g = step_calls(binding, mode_name, dev, bufs, T, h, f, t, ws, None)
 
         def step_current_stream():
             for c in calls_g:
@@ -774,7 +790,7 @@ def main():
         binding.mlp_tp_check(ws, sh)
         ms_g, fl_g = reduce_max_sum(s_g.elapsed_time(e_g), float(wl.flops) * n_g)
         graph = {"value": fl_g / (ms_g * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_g / n_g, "steps": n_g,
-                 "api": "the stage calls of one step captured once in a CUDA graph and replayed"}
+                 "api": "mlp_tp_forward + mlp_tp_backward of one step captured once in a CUDA graph and replayed"}
         del cg
 
     # ------------------------------------------------ activation recomputation

@@ -51,10 +51,14 @@
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *    enqueued on it; no entry point except mlp_tp_check synchronises, and
  *    none allocates or frees memory.  The enqueued work is kernel launches
- *    and asynchronous memsets only, so a sequence of calls can be captured
- *    into a CUDA graph and replayed (after one uncaptured call per shape,
- *    which sets the kernels' shared-memory limits); a replay reads the
- *    buffers' current contents.
+ *    and asynchronous memsets; in addition, mlp_tp_forward / mlp_tp_backward
+ *    (and the recomputing pair) in MLP_TP_FP8 run the mode's operand copies
+ *    on a second stream the library owns (one per device and host thread,
+ *    created on first use), forked from and joined back into `stream` with
+ *    events, so stream order holds for the caller.  A sequence of calls can
+ *    be captured into a CUDA graph and replayed (after one uncaptured call
+ *    per shape, which sets the kernels' shared-memory limits and creates that
+ *    stream); a replay reads the buffers' current contents.
  *  - Results are reproducible bit for bit for a given GPU model, shape and
  *    t: every reduction runs in a fixed order.
  *  - Arguments are validated on the host before anything is launched; on any

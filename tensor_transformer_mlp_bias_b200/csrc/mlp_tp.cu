@@ -829,8 +829,9 @@ mlp_status_t fp8_prepare_forward(const Shape& s, const void* B, const Fp8Bufs& q
 
 // Statistics of X, dY and B, then X -> (X16, X8), dY -> (dY16, dY8) and
 // A -> W16.
-mlp_status_t fp8_prepare_backward(const Shape& s, const void* dY, const void* X, const void* A, const void* B,
-                                  const Fp8Bufs& q, void* ws, const Launch& L) {
+// The statistics of X, dY and B (the scales follow from them).
+mlp_status_t fp8_backward_stats(const Shape& s, const void* dY, const void* X, const void* B, const Fp8Bufs& q,
+                                const Launch& L) {
   mlp_status_t st = zero_fill(q.stats, STAT_WORDS * sizeof(unsigned int), L.stream, "cudaMemsetAsync(fp8 statistics)");
   if (st != MLP_OK) return st;
   const long long rows = 2LL * s.T + s.f;
@@ -842,16 +843,79 @@ mlp_status_t fp8_prepare_backward(const Shape& s, const void* dY, const void* X,
                                 static_cast<int>(s.f), q.stats);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_stats");
   g_launches.fetch_add(1);
+  return MLP_OK;
+}
+
+// dY -> (dY16, dY8), A -> W16, X -> (X16, X8), in the order the backward
+// GEMMs need them; after fp8_backward_stats.
+mlp_status_t fp8_backward_casts(const Shape& s, const void* dY, const void* X, const void* A, const Fp8Bufs& q,
+                                void* ws, const Launch& L) {
   CastJobs jobs;
   memset(&jobs, 0, sizeof(jobs));
-  jobs.job[0] = CastJob{static_cast<const __nv_bfloat16*>(X), static_cast<__half*>(q.x16),
-                        static_cast<uint8_t*>(q.x8), s.T * s.h, CAST_SX};
-  jobs.job[1] = CastJob{static_cast<const __nv_bfloat16*>(dY), static_cast<__half*>(q.dy16),
+  jobs.job[0] = CastJob{static_cast<const __nv_bfloat16*>(dY), static_cast<__half*>(q.dy16),
                         static_cast<uint8_t*>(q.dy8), s.T * s.h, CAST_SY};
-  jobs.job[2] = CastJob{static_cast<const __nv_bfloat16*>(A), static_cast<__half*>(q.w16), nullptr, s.h * s.f,
+  jobs.job[1] = CastJob{static_cast<const __nv_bfloat16*>(A), static_cast<__half*>(q.w16), nullptr, s.h * s.f,
                         CAST_UNSCALED};
+  jobs.job[2] = CastJob{static_cast<const __nv_bfloat16*>(X), static_cast<__half*>(q.x16),
+                        static_cast<uint8_t*>(q.x8), s.T * s.h, CAST_SX};
   jobs.count = 3;
   return launch_cast(jobs, q.stats, ws, L);
+}
+
+// Statistics, then the copies, on one stream.
+mlp_status_t fp8_prepare_backward(const Shape& s, const void* dY, const void* X, const void* A, const void* B,
+                                  const Fp8Bufs& q, void* ws, const Launch& L) {
+  mlp_status_t st = fp8_backward_stats(s, dY, X, B, q, L);
+  return st != MLP_OK ? st : fp8_backward_casts(s, dY, X, A, q, ws, L);
+}
+
+// A second stream per device and host thread for the fp8 mode's operand
+// copies inside the composite calls.  The copies are HBM-bound and the GEMMs
+// leave most of the HBM bandwidth and room for one more small block on each
+// SM, so running them beside the GEMMs hides them.  The fork and the join are
+// events: the side stream waits for everything enqueued before the fork, and
+// the GEMM that reads the copies waits for the join, so stream order is kept
+// for the caller (and a CUDA graph capture follows the fork and the join).
+// Created on first use with the device current; never destroyed.
+struct SideLane {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+thread_local SideLane g_side[64];
+
+mlp_status_t side_lane(int dev, SideLane** out) {
+  SideLane& l = g_side[dev];
+  if (l.stream == nullptr) {
+    cudaError_t e = cudaStreamCreateWithFlags(&l.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "creating the fp8 mode's side stream");
+  }
+  *out = &l;
+  return MLP_OK;
+}
+
+// The side stream waits for the work enqueued on L.stream so far; returns the
+// launch description of the side stream.
+mlp_status_t fork_side(const Launch& L, SideLane** lane, Launch* side) {
+  mlp_status_t st = side_lane(L.dev, lane);
+  if (st != MLP_OK) return st;
+  cudaError_t e = cudaEventRecord((*lane)->fork, L.stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent((*lane)->stream, (*lane)->fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "forking the fp8 mode's side stream");
+  *side = L;
+  side->stream = (*lane)->stream;
+  return MLP_OK;
+}
+
+mlp_status_t record_join(SideLane* lane) {
+  cudaError_t e = cudaEventRecord(lane->join, lane->stream);
+  return e == cudaSuccess ? MLP_OK : cuda_fail(e, "joining the fp8 mode's side stream");
+}
+
+mlp_status_t wait_join(SideLane* lane, const Launch& L) {
+  cudaError_t e = cudaStreamWaitEvent(L.stream, lane->join, 0);
+  return e == cudaSuccess ? MLP_OK : cuda_fail(e, "joining the fp8 mode's side stream");
 }
 
 Operand op16(const void* p, bool mn) { return Operand{{p, p}, mn, {OP_F16, OP_F16}}; }
@@ -968,8 +1032,17 @@ mlp_status_t backward_fp8(const Shape& s, const void* dY, const void* X, const v
   void* dH16 = static_cast<char*>(ws) + dh_offset();
   void* dH8 = static_cast<char*>(ws) + dh_lo_offset(s);
   mlp_status_t st;
-  if ((st = fp8_prepare_backward(s, dY, X, A, B, q, ws, L)) != MLP_OK) return st;
+  // statistics first (every scale needs them), then the copies on the side
+  // stream beside the GeLU-derivative GEMM, joined before the first GEMM that
+  // reads them (dB)
+  SideLane* lane = nullptr;
+  Launch side;
+  if ((st = fp8_backward_stats(s, dY, X, B, q, L)) != MLP_OK) return st;
+  if ((st = fork_side(L, &lane, &side)) != MLP_OK) return st;
+  if ((st = fp8_backward_casts(s, dY, X, A, q, ws, side)) != MLP_OK) return st;
+  if ((st = record_join(lane)) != MLP_OK) return st;
   if ((st = fc2_backward_data_fp8(s, dY, B, Z, dH16, dH8, da, q.stats, ws, L)) != MLP_OK) return st;
+  if ((st = wait_join(lane, L)) != MLP_OK) return st;
   if ((st = fc2_backward_weight_fp8(s, H16, H8, q.dy16, q.dy8, dY, dB, db, q.stats, ws, L)) != MLP_OK) return st;
   if ((st = fc1_backward_data_fp8(s, dH16, q.w16, dX, q.stats, ws, L)) != MLP_OK) return st;
   return fc1_backward_weight_fp8(s, q.x16, q.x8, dH16, dH8, dA, q.stats, ws, L);
@@ -979,8 +1052,14 @@ mlp_status_t forward_fp8(const Shape& s, const void* X, const void* A, const voi
                          void* Y, void* Z, void* H16, void* H8, void* ws, bool recompute, const Launch& L) {
   const Fp8Bufs q = fp8_bufs(ws, s, recompute);
   mlp_status_t st;
-  if ((st = fp8_prepare_forward(s, B, q, ws, L)) != MLP_OK) return st;
+  // the fp16 copy of B on the side stream beside the column-parallel GEMM
+  SideLane* lane = nullptr;
+  Launch side;
+  if ((st = fork_side(L, &lane, &side)) != MLP_OK) return st;
+  if ((st = fp8_prepare_forward(s, B, q, ws, side)) != MLP_OK) return st;
+  if ((st = record_join(lane)) != MLP_OK) return st;
   if ((st = fc1_forward_fp8(s, X, A, a, Z, H16, H8, ws, L)) != MLP_OK) return st;
+  if ((st = wait_join(lane, L)) != MLP_OK) return st;
   return fc2_forward_fp8(s, H16, q.w16, b, Y, ws, L);
 }
 
