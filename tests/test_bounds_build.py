@@ -8,7 +8,8 @@ outside it.  It stands in for a memory checker, which this machine does not
 offer.  The shapes below reach every checked site: split shard-sum tails,
 K-split weight gradients, ragged tiles, da and db, a batch whose [T, f]
 tensors hold more than 2^31 elements, the allocation-free path, and the
-cross-GPU path's peer stores and reduce (two ranks emulated on this GPU).  They must pass with a clean status
+cross-GPU path's peer stores and reduce (two ranks emulated on this GPU), and
+the fp16 + e4m3 mode.  They must pass with a clean status
 word and meet the parity bar.
 """
 import os
@@ -32,7 +33,9 @@ from oracle import mlp_oracle as oracle
 from tensor_transformer_mlp_bias_b200 import block, inputs
 from tests.parity_util import assert_close, to_gpu
 shapes = [(333, 320, 1280, 5, 3), (1024, 256, 1024, 2, 3), (2048, 128, 512, 4, 0), (1, 64, 128, 2, 3),
-          (257, 512, 768, 3, 0)]
+          (257, 512, 768, 3, 0),
+          # the fp16 + e4m3 mode: casts, statistics, the e4m3 stages' ragged token tail, K-split pieces
+          (333, 320, 1280, 5, 4), (1024, 256, 1024, 2, 4), (129, 192, 768, 3, 4)]
 for T, h, f, t, mode in shapes:
     inp = inputs.make_custom(T, h, f, seed=T + f)
     out = block.forward_backward(to_gpu(inp), t, mode=mode)  # mlp_tp_check raises on MLP_ERR_BOUNDS
@@ -56,6 +59,14 @@ assert_close("dX rows", out["dX"][r], sr["dX"])
 assert_close("dA cols", out["dA"][:, c], sc["dA"])
 assert_close("dB rows", out["dB"][c, :], sc["dB"])
 assert_close("da cols", out["da"][c], sc["da"])
+del out
+torch.cuda.empty_cache()
+# the same batch in the fp16 + e4m3 mode (e4m3 [T, f] tensors of 2.18e9 bytes)
+out = block.forward_backward(to_gpu(inp), t, mode=binding.FP8)
+assert_close("Y rows (fp8)", out["Y"][r], sr["Y"])
+assert_close("dX rows (fp8)", out["dX"][r], sr["dX"])
+assert_close("dA cols (fp8)", out["dA"][:, c], sc["dA"])
+assert_close("dB rows (fp8)", out["dB"][c, :], sc["dB"])
 del out, inp
 torch.cuda.empty_cache()
 T, h = 4096, 1024
