@@ -920,7 +920,8 @@ def main():
     # ------------------------------------------------ roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     roofline = roofline_entry(stage_ms, mode, T, h, f, clk_stages.summary(), peaks, peak_src)
-    roofline["traffic"] = traffic_for(roofline["stage"], wl, t) if args.tokens is None else None
+    prefix = "fp8." if mode_name == "fp8" else ""  # the table keys the fp8 mode's kernels apart
+    roofline["traffic"] = traffic_for(prefix + roofline["stage"], wl, t) if args.tokens is None else None
     products = stage_products(mode)
     clocks = clk.summary()
     peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))

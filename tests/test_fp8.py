@@ -242,3 +242,23 @@ def test_binding_refuses_bf16_activations_in_fp8_calls():
     Y = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError):
         binding.mlp_tp_fc2_forward_fp8(Hb, inp["b"], T, h, f, t, Y, ws)
+
+
+def _random_shapes(n=10, seed=2025):
+    """Ragged token counts (not multiples of the 128-token e4m3 stage), hidden sizes and shard widths."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        t = int(rng.integers(1, 9))
+        fs = 64 * int(rng.integers(1, 7))
+        h = 64 * int(rng.integers(1, 11))
+        T = int(rng.integers(1, 900))
+        out.append((T, h, fs * t, t))
+    return out
+
+
+@pytest.mark.parametrize("shape", _random_shapes(), ids=lambda s: "T%d_h%d_f%d_t%d" % s)
+def test_random_shapes_full_oracle(shape):
+    T, h, f, t = shape
+    inp = inputs.make_custom(T, h, f, seed=T * 5 + h + f + t)
+    check_full(run_fp8(to_gpu(inp), t), oracle.full(inp))
