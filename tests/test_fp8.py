@@ -68,8 +68,9 @@ def test_tiny_workload_every_divisor():
         check_full(run_fp8(g, t), ref)
 
 
-@pytest.mark.parametrize("t", [1, 8])
+@pytest.mark.parametrize("t", [1, 8, 64])
 def test_gpt2_medium_full_oracle(t):
+    """t = 64: shards of 64 columns, the narrowest allowed (one K slice per shard segment of Y and dX)."""
     inp, ref = _gpt2_medium()
     check_full(run_fp8(to_gpu(inp), t), ref)
 
