@@ -263,3 +263,18 @@ def test_random_shapes_full_oracle(shape):
     T, h, f, t = shape
     inp = inputs.make_custom(T, h, f, seed=T * 5 + h + f + t)
     check_full(run_fp8(to_gpu(inp), t), oracle.full(inp))
+
+
+def test_weight_beyond_fp16_is_reported():
+    """A weight fp16 cannot hold (|w| > 65504, fine in bf16) makes the fp16 copy of B infinite; the cast
+    records MLP_ERR_RANGE instead of the step failing silently."""
+    T, h, f, t = 128, 128, 512, 2
+    host = inputs.make_custom(T, h, f, seed=45)
+    host["B"][3, 7] = 1.0e5
+    inp = to_gpu(host)
+    out = block.alloc_outputs(T, h, f, mode=FP8)
+    ws = binding.make_workspace_mode(T, h, f, t, FP8)
+    block.forward(inp, t, out, ws, FP8)
+    with pytest.raises(binding.MlpError) as err:
+        binding.mlp_tp_check(ws)
+    assert err.value.status == 9
