@@ -54,7 +54,8 @@ static int to_file(const char* path, const void* d, size_t bytes) {
 }
 
 int main(int argc, char** argv) {
-  if (argc != 7) return 2;
+  if (argc != 8) return 2;
+  const int mode = std::atoi(argv[7]);  // MLP_TP_ACCURATE, or MLP_TP_FP8 (H then holds fp16 values)
   const int64_t T = std::atoll(argv[1]), h = std::atoll(argv[2]), f = std::atoll(argv[3]);
   const int32_t t = std::atoi(argv[4]);
   const char* in_path = argv[5];
@@ -80,14 +81,14 @@ int main(int argc, char** argv) {
   CK(cudaMalloc(&da, f * b2));
   CK(cudaMalloc(&dB, f * h * b2));
   CK(cudaMalloc(&db, h * b2));
-  const size_t ws_bytes = mlp_tp_workspace_bytes(T, h, f, t);
+  const size_t ws_bytes = mlp_tp_workspace_bytes_mode(T, h, f, t, mode);
   if (ws_bytes == 0) return 5;
   CK(cudaMalloc(&ws, ws_bytes));
   CK(cudaMemset(ws, 0, ws_bytes));
   cudaStream_t s;
   CK(cudaStreamCreate(&s));
-  MK(mlp_tp_forward(X, A, a, B, b, T, h, f, t, MLP_TP_ACCURATE, Y, Z, H, H_lo, ws, ws_bytes, s));
-  MK(mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, MLP_TP_ACCURATE, dX, dA, da, dB, db, ws, ws_bytes, s));
+  MK(mlp_tp_forward(X, A, a, B, b, T, h, f, t, mode, Y, Z, H, H_lo, ws, ws_bytes, s));
+  MK(mlp_tp_backward(dY, X, A, B, Z, H, H_lo, T, h, f, t, mode, dX, dA, da, dB, db, ws, ws_bytes, s));
   MK(mlp_tp_check(ws, s));
   char p[4096];
   const char* names[] = {"Y", "Z", "H", "dX", "dA", "da", "dB", "db"};
@@ -115,7 +116,8 @@ def _load(path, shape, f32=False):
     return (raw.astype(np.uint32) << 16).view(np.float32).reshape(shape).astype(np.float64)
 
 
-def test_cpp_client_runs_the_block_through_the_c_abi(tmp_path):
+@pytest.mark.parametrize("mode", [0, 4], ids=["accurate", "fp8"])
+def test_cpp_client_runs_the_block_through_the_c_abi(tmp_path, mode):
     gxx = shutil.which("g++")
     if gxx is None or not os.path.exists(os.path.join(CUDA, "include", "cuda_runtime.h")):
         pytest.skip("g++ or the CUDA headers are not available")
@@ -139,7 +141,7 @@ def test_cpp_client_runs_the_block_through_the_c_abi(tmp_path):
             fh.write(_bf16_bytes(inp[k]))
     out_dir = tmp_path / "out"
     out_dir.mkdir()
-    run = subprocess.run([str(exe), str(T), str(h), str(f), str(t), str(blob), str(out_dir)],
+    run = subprocess.run([str(exe), str(T), str(h), str(f), str(t), str(blob), str(out_dir), str(mode)],
                          capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert int(run.stdout.split()[-1]) > 0  # the library's own kernels ran
@@ -148,5 +150,8 @@ def test_cpp_client_runs_the_block_through_the_c_abi(tmp_path):
     shapes = {"Y": (T, h), "Z": (T, f), "H": (T, f), "dX": (T, h), "dA": (h, f), "da": (f,), "dB": (f, h),
               "db": (h,)}
     for k, shp in shapes.items():
-        got = _load(out_dir / f"{k}.bin", shp, f32=(k == "Z"))
+        if k == "H" and mode == 4:  # the fp8 mode's H is fp16 (its e4m3 residual stays on the device)
+            got = np.fromfile(out_dir / "H.bin", dtype=np.float16).reshape(shp).astype(np.float64)
+        else:
+            got = _load(out_dir / f"{k}.bin", shp, f32=(k == "Z"))
         assert_close(k + " (C++ client)", got, ref[k])
