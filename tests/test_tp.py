@@ -91,8 +91,9 @@ def test_two_ranks_match_the_unsharded_block(sp, mode):
             assert e < 1e-12, (rank, k, e)
 
 
-def test_four_ranks_sequence_parallel_match_the_unsharded_block():
-    res = _run(4, (64, 128, 512), True, 0)
+@pytest.mark.parametrize("mode", [0, 4], ids=["accurate", "fp8"])
+def test_four_ranks_sequence_parallel_match_the_unsharded_block(mode):
+    res = _run(4, (64, 128, 512), True, mode)
     assert set(res) == {0, 1, 2, 3}
     for rank, errs in res.items():
         for k, e in errs.items():
