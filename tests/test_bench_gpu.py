@@ -1,6 +1,6 @@
 """bench.py's JSON line on the GPU: one short run of the tiny workload in a
-subprocess, checked key by key against the contract the harness
-reads (metric, value, ms_per_step, steps, warmup, roofline, e2e with the
+subprocess, checked key by key against the contract its consumers
+read (metric, value, ms_per_step, steps, warmup, roofline, e2e with the
 bytes it copies, clocks, gpu_launches) and for internal consistency (value
 against ms_per_step and the workload's FLOPs, frac against achieved and peak,
 the launch count against the steps)."""
