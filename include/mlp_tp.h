@@ -243,7 +243,9 @@ mlp_status_t mlp_tp_fc1_backward_weight(const void* X, const void* dH, const voi
  * backward of mlp_tp_backward.  Both need
  * mlp_tp_recompute_workspace_bytes(T, h, f, t) bytes of workspace (the
  * ordinary workspace plus T·f·8 bytes for Z, H, H_lo).  Same conventions
- * and modes as mlp_tp_forward / mlp_tp_backward. */
+ * and modes as mlp_tp_forward / mlp_tp_backward; with MLP_TP_FP8 the
+ * workspace is mlp_tp_recompute_workspace_bytes_mode(..., MLP_TP_FP8)
+ * bytes (the mode's operand copies after the recomputed activations). */
 size_t mlp_tp_recompute_workspace_bytes(int64_t T, int64_t h, int64_t f, int32_t t);
 size_t mlp_tp_recompute_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode);
 
