@@ -278,3 +278,22 @@ def test_weight_beyond_fp16_is_reported():
     with pytest.raises(binding.MlpError) as err:
         binding.mlp_tp_check(ws)
     assert err.value.status == 9
+
+
+def test_t_independence_and_determinism():
+    """As in the bf16 modes: Z, H, H_lo, dA, dB, da, db do not depend on t bit for bit (the scales follow from
+    statistics over whole tensors, not shards), Y and dX only through the shard-sum order, and a rerun
+    (statistics by atomic max, copies on the side stream) gives the same bits."""
+    T, h, f = 384, 512, 2048
+    inp = to_gpu(inputs.make_custom(T, h, f, seed=5))
+    outs = {t: run_fp8(inp, t) for t in (1, 2, 4, 8)}
+    same = lambda a, b: torch.equal(a.view(torch.uint8), b.view(torch.uint8))  # noqa: E731
+    for t in (2, 4, 8):
+        for k in ("Z", "H", "H_lo", "dA", "dB", "da", "db"):
+            assert same(outs[t][k], outs[1][k]), (k, t)
+        for k in ("Y", "dX"):
+            d = (outs[t][k].float() - outs[1][k].float()).abs()
+            assert float(d.max()) <= 1e-2 * (1 + float(outs[1][k].float().abs().max())), (k, t)
+    again = run_fp8(inp, 8)
+    for k in again:
+        assert same(again[k], outs[8][k]), k
