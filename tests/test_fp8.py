@@ -297,3 +297,31 @@ def test_t_independence_and_determinism():
     again = run_fp8(inp, 8)
     for k in again:
         assert same(again[k], outs[8][k]), k
+
+
+def test_outputs_stay_inside_their_buffers():
+    """Guard bands around every output and saved activation, with a ragged shape: the fp16 and e4m3 tiles'
+    stores (32-byte rows for e4m3) are clipped at the tensors' edges."""
+    T, h, f, t = 200, 192, 384, 3
+    inp = to_gpu(inputs.make_custom(T, h, f, seed=4))
+    shapes = {"Y": (T, h), "Z": (T, f), "H": (T, f), "H_lo": (T, f), "dX": (T, h), "dA": (h, f), "dB": (f, h),
+              "da": (f,), "db": (h,)}
+    dtypes = {"Z": torch.float32, "H": torch.float16, "H_lo": torch.uint8}
+    pad = 4096
+    bufs, out = {}, {}
+    for k, s in shapes.items():
+        n = int(np.prod(s))
+        buf = torch.full((n + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda") if k == "H_lo" else \
+            torch.full((n + 2 * pad,), -12345.0, dtype=dtypes.get(k, torch.bfloat16), device="cuda")
+        bufs[k] = buf
+        out[k] = buf[pad:pad + n].view(*s)
+    ws = binding.make_workspace_mode(T, h, f, t, FP8)
+    block.forward(inp, t, out, ws, FP8)
+    block.backward(inp, t, out, ws, FP8)
+    binding.mlp_tp_check(ws)
+    for k, buf in bufs.items():
+        n = int(np.prod(shapes[k]))
+        head, tail = buf[:pad].cpu(), buf[pad + n:].cpu()
+        assert torch.equal(head, torch.full_like(head, head[0])) and torch.equal(tail, torch.full_like(tail, head[0])), k
+    out["H_lo"] = out["H_lo"].view(torch.float8_e4m3fn)
+    check_full(out, oracle.full(inputs.make_custom(T, h, f, seed=4)))
