@@ -159,8 +159,9 @@ size_t mlp_tp_workspace_bytes_mode(int64_t T, int64_t h, int64_t f, int32_t t, i
 /* ---------------------------------------------------------------- forward */
 
 /* Whole forward: mlp_tp_fc1_forward then mlp_tp_fc2_forward (the latter
- * given H_lo unless `mode` has MLP_TP_FAST_FC2_FORWARD).  Writes Y[T,h] and
- * saves Z[T,f] (fp32), H[T,f] and H_lo[T,f] for the backward. */
+ * given H_lo unless `mode` has MLP_TP_FAST_FC2_FORWARD; with MLP_TP_FP8 the
+ * fp8 calls below).  Writes Y[T,h] and saves Z[T,f] (fp32), H[T,f] and
+ * H_lo[T,f] for the backward. */
 mlp_status_t mlp_tp_forward(const void* X, const void* A, const void* a,
                             const void* B, const void* b,
                             int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
@@ -190,8 +191,9 @@ mlp_status_t mlp_tp_fc2_forward(const void* H, const void* H_lo, const void* B, 
 /* Whole backward, given dY and Z, H, H_lo saved by the forward:
  * mlp_tp_fc2_backward_data (dH pair into the workspace),
  * mlp_tp_fc2_backward_weight, mlp_tp_fc1_backward_data (given dH_lo unless
- * `mode` has MLP_TP_FAST_FC1_BACKWARD_DATA) and mlp_tp_fc1_backward_weight.
- * `da` and `db` may be NULL (bias gradients not wanted). */
+ * `mode` has MLP_TP_FAST_FC1_BACKWARD_DATA) and mlp_tp_fc1_backward_weight;
+ * with MLP_TP_FP8 the fp8 calls below.  `da` and `db` may be NULL (bias
+ * gradients not wanted). */
 mlp_status_t mlp_tp_backward(const void* dY, const void* X, const void* A,
                              const void* B, const void* Z, const void* H, const void* H_lo,
                              int64_t T, int64_t h, int64_t f, int32_t t, int32_t mode,
@@ -265,7 +267,9 @@ mlp_status_t mlp_tp_backward_recompute(const void* dY, const void* X, const void
 
 /* The stages of MLP_TP_FP8 (see the mode's description above), for callers
  * that interleave other work; mlp_tp_forward / mlp_tp_backward with
- * MLP_TP_FP8 are exactly these calls in this order.  All of them take a
+ * MLP_TP_FP8 run the same kernels in this order and give the same bits (they
+ * only move the casts of the prepare calls onto their side stream, beside
+ * the GEMMs).  All of them take a
  * workspace of mlp_tp_workspace_bytes_mode(..., MLP_TP_FP8) bytes, and the
  * same workspace from the prepare call on:
  *   forward:  mlp_tp_fp8_prepare_forward (fp16 copy of B into the workspace),
