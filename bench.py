@@ -922,6 +922,8 @@ def main():
     roofline = roofline_entry(stage_ms, mode, T, h, f, clk_stages.summary(), peaks, peak_src)
     prefix = "fp8." if mode_name == "fp8" else ""  # the table keys the fp8 mode's kernels apart
     roofline["traffic"] = traffic_for(prefix + roofline["stage"], wl, t) if args.tokens is None else None
+    if mode_name == "accurate" and roofline["stage"] in ("fc2_forward", "fc1_backward_data"):
+        roofline["traffic"] = None  # the table holds the fast mode's one-half form of these two GEMMs
     products = stage_products(mode)
     clocks = clk.summary()
     peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
